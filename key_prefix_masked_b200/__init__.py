@@ -1,0 +1,33 @@
+"""B200-native (sm_100a) prefix-masked attention forward.
+
+    out, lse = attn_prefix_fwd(q, k, v, kv_len)          # single pass
+    out, lse = attn_prefix_fwd_splitkv(q, k, v, kv_len, num_splits=64)
+
+q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 256}; kv_len:
+int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never take part).
+The computation runs in the hand-written kernels of the C library built from csrc/;
+this package only marshals arguments.
+"""
+from ._binding import (  # noqa: F401
+    AttnError,
+    ATTN_OK,
+    ATTN_ERR_INVALID_ARG,
+    ATTN_ERR_UNSUPPORTED,
+    ATTN_ERR_CUDA,
+    ATTN_ERR_TIMEOUT,
+    ATTN_ERR_KVLEN_RANGE,
+    ATTN_DEBUG_DROP_COPY,
+    SUPPORTED_HEAD_DIMS,
+    LIB_PATH,
+    device_status,
+    fwd as attn_prefix_fwd,
+    fwd_split as attn_prefix_fwd_split,
+    fwd_splitkv as attn_prefix_fwd_splitkv,
+    lib,
+    lse_combine as attn_lse_combine,
+    set_debug_flags,
+    set_wait_limit_ns,
+    split_chunk_len,
+    status_string,
+    version,
+)

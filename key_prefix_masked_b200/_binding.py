@@ -1,0 +1,186 @@
+"""ctypes binding of the C ABI declared in include/attn_prefix.h.
+
+Argument marshalling only: torch provides device memory and the current stream; every
+step of the computation runs in the library's sm_100a kernels.  If the compiled library
+is missing, importing the functions raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_build", "libattn_prefix.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+ATTN_ERR_KVLEN_RANGE = 5
+ATTN_DEBUG_DROP_COPY = 1
+
+SUPPORTED_HEAD_DIMS = (32, 64, 256)
+
+# Every symbol the header exports, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SIGNATURES = {
+    "attn_prefix_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "attn_split_chunk_len": (_I, [_I, _I]),
+    "attn_split_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_split_lse_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_prefix_fwd_split": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "attn_lse_combine": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_get_device_status": (_I, [_P]),
+    "attn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+    "attn_set_debug_flags": (None, [ctypes.c_uint]),
+    "attn_status_string": (ctypes.c_char_p, [_I]),
+    "attn_version": (_I, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"CUDA library not built: {LIB_PATH} is missing "
+                    "(run `python -m key_prefix_masked_b200.build` or __graft_entry__.build())")
+            handle = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _check_qkv(q, k, v, kv_len):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B,H,T,D]")
+    B, H, Tq, D = q.shape
+    if k.shape[:2] != (B, H) or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError("k and v must be [B,H,Tk,D] matching q's B, H, D")
+    if (not kv_len.is_cuda or kv_len.dtype != torch.int32 or kv_len.numel() != B
+            or not kv_len.is_contiguous()):
+        raise ValueError("kv_len must be a contiguous int32 CUDA tensor of B entries")
+    if len({q.device, k.device, v.device, kv_len.device}) != 1:
+        raise ValueError("all tensors must be on one device")
+    return int(B), int(H), int(Tq), int(k.shape[2]), int(D)
+
+
+def fwd(q, k, v, kv_len, scale=None, out=None, lse=None, need_lse=True):
+    """Prefix-masked attention forward (attn_prefix_fwd): returns (out bf16, lse fp32)."""
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib().attn_prefix_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), _ptr(out), _ptr(lse),
+                                   B, H, Tq, Tk, D, scale, _stream_ptr(q.device))
+    _check(st, "attn_prefix_fwd")
+    return out, lse
+
+
+def split_chunk_len(Tk: int, num_splits: int) -> int:
+    return int(lib().attn_split_chunk_len(int(Tk), int(num_splits)))
+
+
+def fwd_split(q, k, v, kv_len, num_splits, scale=None, part_out=None, part_lse=None):
+    """Split-KV partials (attn_prefix_fwd_split): fp32 part_out [C,B,H,Tq,D], part_lse [C,B,H,Tq]."""
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len)
+    C = int(num_splits)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if part_out is None:
+        part_out = torch.empty((C, B, H, Tq, D), dtype=torch.float32, device=q.device)
+    if part_lse is None:
+        part_lse = torch.empty((C, B, H, Tq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib().attn_prefix_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), C, _ptr(part_out),
+                                         _ptr(part_lse), B, H, Tq, Tk, D, scale,
+                                         _stream_ptr(q.device))
+    _check(st, "attn_prefix_fwd_split")
+    return part_out, part_lse
+
+
+def lse_combine(part_out, part_lse, out=None, lse=None, need_lse=True):
+    """Exact LSE combination of split partials (attn_lse_combine): (out bf16, lse fp32)."""
+    if part_out.dtype != torch.float32 or part_lse.dtype != torch.float32:
+        raise ValueError("partials must be fp32")
+    if not (part_out.is_contiguous() and part_lse.is_contiguous()):
+        raise ValueError("partials must be contiguous")
+    C, B, H, Tq, D = (int(s) for s in part_out.shape)
+    if tuple(part_lse.shape) != (C, B, H, Tq):
+        raise ValueError("part_lse must be [C,B,H,Tq]")
+    if out is None:
+        out = torch.empty((B, H, Tq, D), dtype=torch.bfloat16, device=part_out.device)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=part_out.device)
+    with torch.cuda.device(part_out.device):
+        st = lib().attn_lse_combine(_ptr(part_out), _ptr(part_lse), C, _ptr(out), _ptr(lse),
+                                    B, H, Tq, D, _stream_ptr(part_out.device))
+    _check(st, "attn_lse_combine")
+    return out, lse
+
+
+def fwd_splitkv(q, k, v, kv_len, num_splits, scale=None, workspace=None):
+    """Split-KV forward: partials over num_splits key chunks, then the LSE combine."""
+    part_out, part_lse = fwd_split(q, k, v, kv_len, num_splits, scale,
+                                   *(workspace if workspace is not None else (None, None)))
+    return lse_combine(part_out, part_lse)
+
+
+def device_status(device=None) -> int:
+    """Synchronizes the current stream and returns (and clears) the sticky device flags."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib().attn_get_device_status(_stream_ptr(dev)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().attn_set_wait_limit_ns(int(ns))
+
+
+def set_debug_flags(flags: int) -> None:
+    lib().attn_set_debug_flags(int(flags))
+
+
+def version() -> int:
+    return int(lib().attn_version())

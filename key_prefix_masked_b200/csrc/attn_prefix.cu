@@ -1,0 +1,824 @@
+// attn_prefix.cu -- B200 (sm_100a) prefix-masked attention forward: kernels and C ABI.
+//
+// The operation (declared in include/attn_prefix.h) is scaled-dot-product attention in
+// which batch element b sees only its first kv_len[b] keys.  That is the boolean
+// [B,1,1,Tk] key-prefix mask of "Rewrite prefix key-padding masks as k/v truncation to
+// keep SDPA on the flash path" ("Problem", "Fix"), which equals truncating k/v to the
+// valid rows, carried as a per-batch count like the key_value_seq_lengths of "Add
+// sequence-parallel multi-GPU inference ... and a cuDNN flash attention option" ("cuDNN
+// flash attention").  The softmax is an fp32 online softmax that also emits the per-row
+// log-sum-exp, so partial results over key chunks combine exactly ("Sequence-parallel
+// inference" on the same page): attn_prefix_fwd_split + attn_lse_combine.
+//
+// Kernel design (one CTA = one 128-row query tile of one (b, h), optionally one key
+// chunk; 6 warps):
+//   warp 4      TMA producer: Q tile once, then K and V chunks into a ring of 16 KB
+//               shared-memory slots, in exactly the order the MMA warp consumes them.
+//               Key tiles at or beyond kv_len are never requested.
+//   warp 5      MMA issuer (one thread): S_j = Q K_j^T with both operands in shared
+//               memory into a double-buffered fp32 TMEM tile (128 x 128), and
+//               O += P_j V_j with P read from TMEM (bf16, written over S_j) and V from
+//               shared memory into an fp32 TMEM accumulator (128 x D).  It also owns
+//               the TMEM allocation.
+//   warps 0-3   softmax + epilogue: thread t owns query row t (TMEM lane t).  Scores of
+//               keys >= kv_len are replaced by -inf by selection; the running max is
+//               kept in the log2 domain and O is rescaled in TMEM only when the max grows
+//               by more than 2^8 (exact either way: O and the row sum always share one
+//               reference max).  At the end O is divided by the row sum and written as
+//               bf16 (fp32 for split partials) with lse = ln(sum) + max.
+// In the last, partial key tile the value rows between kv_len and the next multiple of
+// 16 are zeroed in shared memory before the PV MMA, and MMA steps lying wholly past
+// kv_len are skipped, so padding content (NaN included) never reaches an accumulator.
+//
+// Every mbarrier wait is bounded (%globaltimer); on expiry the CTA raises a sticky
+// device flag, drains its copies and MMAs in flight, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "attn_prefix.h"
+#include "ptx.cuh"
+#include "tmem_ops.cuh"
+
+namespace attn {
+
+constexpr int BM = 128;               // query rows per CTA (one TMEM lane each)
+constexpr int BN = 128;               // keys per tile
+constexpr int NUM_THREADS = 192;      // 4 softmax warps + producer warp + MMA warp
+constexpr int SMEM_LIMIT = 232448;    // 227 KB opt-in dynamic shared memory per block
+constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128) S1 [128,256) O [256, 256+D)
+constexpr uint32_t O_COL = 256;
+constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr float LN2 = 0.69314718055994530942f;
+constexpr float LOG2E = 1.44269504088896340736f;
+
+constexpr unsigned STATUS_TIMEOUT = 1u;
+constexpr unsigned STATUS_KVLEN = 2u;
+
+template <int D>
+struct Cfg {
+    static constexpr int SW = (D >= 64) ? 128 : 64;   // swizzle span in bytes
+    static constexpr int BLK = SW / 2;                // bf16 columns per swizzle block
+    static constexpr int NBLK = D / BLK;              // column blocks per row
+    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int SLOT = BN * SW;              // bytes of one K chunk == one V chunk
+    static constexpr int KCH = NBLK;                  // K tile: one chunk per column block
+    static constexpr int VCH = NBLK;                  // V tile: chunks of V_ROWS key rows
+    static constexpr int V_ROWS = BN / VCH;
+    static constexpr int NSLOTS_RAW = (SMEM_LIMIT - Q_BYTES - 2048) / SLOT;
+    static constexpr int NSLOTS = NSLOTS_RAW > 16 ? 16 : NSLOTS_RAW;
+    static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOTS * SLOT + 1024;
+    static constexpr uint32_t LAYOUT = (SW == 128) ? 2u : 4u;
+    static_assert(D % BLK == 0, "head dim must be a multiple of the swizzle block");
+    static_assert(V_ROWS % 16 == 0, "value chunks must hold whole 16-key MMA steps");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+    static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+};
+
+// Barrier slots inside the shared-memory control block.
+enum : int {
+    BAR_Q = 0,
+    BAR_FULL = 1,       // [16] slot filled (TMA tx)
+    BAR_EMPTY = 17,     // [16] slot consumed (tcgen05.commit)
+    BAR_S = 33,         // [2] S_j ready in TMEM buffer j&1
+    BAR_P = 35,         // [2] P_j stored over S_j (128 softmax arrivals)
+    BAR_O = 37,         // [2] PV_j complete (buffer j&1)
+    BAR_DRAIN = 39,
+    NUM_BARS = 40
+};
+
+struct Params {
+    const int32_t* kv_len;
+    __nv_bfloat16* out;   // single pass: bf16 [B,H,Tq,D]
+    float* lse;           // single pass: fp32 [B,H,Tq] or null
+    float* part_out;      // split: fp32 [C,B,H,Tq,D]
+    float* part_lse;      // split: fp32 [C,B,H,Tq]
+    int B, H, Tq, Tk;
+    int n_qtiles;
+    int num_splits;
+    int chunk_len;        // keys per split chunk (multiple of BN)
+    float scale_log2;     // scale * log2(e)
+    unsigned long long wait_ns;
+    unsigned debug;
+};
+
+__device__ unsigned int g_attn_status = 0;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Bounded wait on an mbarrier phase.  Returns false if the CTA's abort flag is set or
+// the time limit runs out (which sets the abort flag and the device timeout flag).
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicOr(&g_attn_status, STATUS_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag: used only to drain work already in flight.
+__device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity,
+                                            unsigned long long limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicOr(&g_attn_status, STATUS_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <int D, bool SPLIT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + C::Q_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::NSLOTS * C::SLOT);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t sQ_addr = smem_u32(sQ);
+    const uint32_t sKV_addr = smem_u32(sKV);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // ---- work unit: query tile fastest, then split chunk, then (b, h)
+    int unit = blockIdx.x;
+    const int qtile = unit % p.n_qtiles;
+    unit /= p.n_qtiles;
+    const int split = SPLIT ? unit % p.num_splits : 0;
+    const int bh = SPLIT ? unit / p.num_splits : unit;
+    const int b = bh / p.H;
+    const int q0 = qtile * BM;
+
+    int kv = __ldg(p.kv_len + b);
+    if (kv < 0 || kv > p.Tk) {
+        if (tid == 0) atomicOr(&g_attn_status, STATUS_KVLEN);
+        kv = kv < 0 ? 0 : p.Tk;
+    }
+    const int k_begin = SPLIT ? split * p.chunk_len : 0;
+    const int k_end = SPLIT ? min(kv, k_begin + p.chunk_len) : kv;
+    const int n_tiles = (k_end > k_begin) ? (k_end - k_begin + BN - 1) / BN : 0;
+
+    if (tid == 0) {
+        mbar_init(BAR(BAR_Q), 1);
+        for (int s = 0; s < 16; ++s) {
+            mbar_init(BAR(BAR_FULL + s), 1);
+            mbar_init(BAR(BAR_EMPTY + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(BAR_S + i), 1);
+            mbar_init(BAR(BAR_P + i), 128);
+            mbar_init(BAR(BAR_O + i), 1);
+        }
+        mbar_init(BAR(BAR_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const unsigned long long wlim = p.wait_ns;
+
+    if (warp == 4) {
+        // ================================================================ producer
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_map(&tm_q);
+            tma_prefetch_map(&tm_k);
+            tma_prefetch_map(&tm_v);
+            mbar_arrive_expect_tx(BAR(BAR_Q), C::Q_BYTES);
+#pragma unroll
+            for (int blk = 0; blk < C::NBLK; ++blk)
+                tma_load_3d(sQ_addr + blk * BM * C::SW, &tm_q, blk * C::BLK, q0, bh, BAR(BAR_Q));
+
+            int slot = 0;
+            uint32_t phase = 0;
+            uint32_t pending = 0, pend_parity = 0;   // per-slot: fill issued, its parity
+            int dropped = -1;
+            bool ok = true;
+            auto next_slot = [&]() {
+                if (++slot == C::NSLOTS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            };
+            auto load_k = [&](int j) {
+                const int key0 = k_begin + j * BN;
+#pragma unroll 1
+                for (int c = 0; c < C::KCH && ok; ++c) {
+                    ok = wait_bar(BAR(BAR_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(BAR(BAR_FULL + slot), C::SLOT);
+                    if ((p.debug & ATTN_DEBUG_DROP_COPY) && j == 0 && c == 0) {
+                        dropped = slot;   // announced but never issued: the consumer times out
+                    } else {
+                        tma_load_3d(sKV_addr + slot * C::SLOT, &tm_k, c * C::BLK, key0, bh,
+                                    BAR(BAR_FULL + slot));
+                        pending |= 1u << slot;
+                        pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
+                    }
+                    next_slot();
+                }
+            };
+            auto load_v = [&](int j) {
+                const int key0 = k_begin + j * BN;
+#pragma unroll 1
+                for (int c = 0; c < C::VCH && ok; ++c) {
+                    ok = wait_bar(BAR(BAR_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(BAR(BAR_FULL + slot), C::SLOT);
+#pragma unroll
+                    for (int blk = 0; blk < C::NBLK; ++blk)
+                        tma_load_3d(sKV_addr + slot * C::SLOT + blk * C::V_ROWS * C::SW, &tm_v,
+                                    blk * C::BLK, key0 + c * C::V_ROWS, bh, BAR(BAR_FULL + slot));
+                    pending |= 1u << slot;
+                    pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
+                    next_slot();
+                }
+            };
+            load_k(0);
+            if (n_tiles > 1) load_k(1);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                load_v(j);
+                if (j + 2 < n_tiles) load_k(j + 2);
+            }
+            if (!ok) {
+                // Drain: every copy issued must land before this CTA's memory is reused.
+                wait_bar_drain(BAR(BAR_Q), 0, wlim);
+                for (int s = 0; s < C::NSLOTS; ++s)
+                    if (((pending >> s) & 1u) && s != dropped)
+                        wait_bar_drain(BAR(BAR_FULL + s), (pend_parity >> s) & 1u, wlim);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ================================================================ MMA issuer
+        if (n_tiles > 0) {
+            constexpr uint32_t IDESC_S = make_idesc_bf16(BM, BN, false);
+            constexpr uint32_t IDESC_PV = make_idesc_bf16(BM, D, true);
+            int slot = 0;
+            uint32_t phase = 0;
+            bool ok = wait_bar(BAR(BAR_Q), 0, abort_flag, wlim);
+            ok = __all_sync(0xffffffffu, ok);
+            auto next_slot = [&]() {
+                if (++slot == C::NSLOTS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            };
+            auto issue_s = [&](int j) {
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+#pragma unroll 1
+                for (int c = 0; c < C::KCH; ++c) {
+                    ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_FULL + slot), phase, abort_flag, wlim));
+                    if (!ok) return;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_base = sQ_addr + c * BM * C::SW;
+                        const uint32_t b_base = sKV_addr + slot * C::SLOT;
+#pragma unroll
+                        for (int kk = 0; kk < C::BLK / 16; ++kk) {
+                            const uint64_t ad = make_smem_desc(a_base + kk * 32, 16, 8 * C::SW, C::LAYOUT);
+                            const uint64_t bd = make_smem_desc(b_base + kk * 32, 16, 8 * C::SW, C::LAYOUT);
+                            mma_ss(d_tmem, ad, bd, IDESC_S, (c | kk) != 0 ? 1u : 0u);
+                        }
+                        tc_commit(BAR(BAR_EMPTY + slot));
+                    }
+                    __syncwarp();
+                    next_slot();
+                }
+                if (lane == 0) tc_commit(BAR(BAR_S + (j & 1)));
+                __syncwarp();
+            };
+            auto issue_pv = [&](int j) {
+                ok = __all_sync(0xffffffffu,
+                                wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+                if (!ok) return;
+                tc_fence_after();
+                const int valid = min(BN, k_end - (k_begin + j * BN));
+                const int kblocks = (valid + 15) >> 4;   // 16-key steps holding a valid key
+                const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+#pragma unroll 1
+                for (int c = 0; c < C::VCH; ++c) {
+                    ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_FULL + slot), phase, abort_flag, wlim));
+                    if (!ok) return;
+                    tc_fence_after();
+                    const uint32_t v_base = sKV_addr + slot * C::SLOT;
+                    // Zero value rows in [valid, 16*kblocks) that fall inside this chunk.
+                    const int r0 = max(valid, c * C::V_ROWS);
+                    const int r1 = min(kblocks * 16, (c + 1) * C::V_ROWS);
+                    if (r1 > r0) {
+                        constexpr int PIECES = C::SW / 16;   // 16-byte pieces per row segment
+                        const int total = (r1 - r0) * C::NBLK * PIECES;
+                        uint8_t* vs = sKV + slot * C::SLOT;
+                        for (int i = lane; i < total; i += 32) {
+                            const int piece = i % PIECES;
+                            const int rb = i / PIECES;
+                            const int blk = rb % C::NBLK;
+                            const int r = r0 + rb / C::NBLK - c * C::V_ROWS;
+                            *reinterpret_cast<uint4*>(vs + blk * C::V_ROWS * C::SW + r * C::SW + piece * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
+                            const int kb = c * (C::V_ROWS / 16) + kk;
+                            if (kb < kblocks) {
+                                const uint64_t bd = make_smem_desc(v_base + kk * 16 * C::SW,
+                                                                   C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
+                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u, bd, IDESC_PV,
+                                       (j == 0 && kb == 0) ? 0u : 1u);
+                            }
+                        }
+                        tc_commit(BAR(BAR_EMPTY + slot));
+                    }
+                    __syncwarp();
+                    next_slot();
+                }
+                if (lane == 0) tc_commit(BAR(BAR_O + (j & 1)));
+                __syncwarp();
+            };
+            if (ok) issue_s(0);
+            if (ok && n_tiles > 1) issue_s(1);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                issue_pv(j);
+                if (ok && j + 2 < n_tiles) issue_s(j + 2);
+            }
+            // Drain: every MMA issued completes before TMEM is released.
+            if (lane == 0) tc_commit(BAR(BAR_DRAIN));
+            __syncwarp();
+            wait_bar_drain(BAR(BAR_DRAIN), 0, wlim);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ softmax
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY;   // reference max, log2 domain
+        float l_sum = 0.0f;        // row sum relative to m_ref
+        bool ok = true;
+#pragma unroll 1
+        for (int j = 0; j < n_tiles; ++j) {
+            ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
+            uint32_t raw[BN];
+            tmem_ld128_wait(s_addr, raw);
+            float x[BN];
+            const int valid = min(BN, k_end - (k_begin + j * BN));
+            float mx = -INFINITY;
+            if (valid >= BN) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    x[c] = __uint_as_float(raw[c]) * sl2;
+                    mx = fmaxf(mx, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    x[c] = (c < valid) ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
+                    mx = fmaxf(mx, x[c]);
+                }
+            }
+            float factor = 1.0f;
+            bool rescale = false;
+            if (j == 0) {
+                m_ref = mx;
+            } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
+                const float m_new = fmaxf(m_ref, mx);
+                factor = fast_exp2(m_ref - m_new);
+                m_ref = m_new;
+                rescale = true;
+            }
+            float tile_sum = 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(x[cc * 32 + 2 * e] - m_ref);
+                    const float p1 = fast_exp2(x[cc * 32 + 2 * e + 1] - m_ref);
+                    tile_sum += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(s_addr + cc * 16, pk);
+            }
+            l_sum = l_sum * factor + tile_sum;
+            if (rescale) {
+                // O may only be touched once PV_{j-1} has completed.
+                ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_O + ((j - 1) & 1)), ((j - 1) >> 1) & 1,
+                                                      abort_flag, wlim));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int oc = 0; oc < D / 32; ++oc) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                    tmem_st32(tmem + lane_base + O_COL + oc * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(BAR_P + (j & 1)));
+        }
+        // ---- epilogue
+        if (ok && n_tiles > 0) {
+            const int jl = n_tiles - 1;
+            ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_O + (jl & 1)), (jl >> 1) & 1, abort_flag, wlim));
+            tc_fence_after();
+        }
+        const int row = q0 + tid;
+        const bool in_range = row < p.Tq;
+        const bool have = n_tiles > 0;
+        const float inv_l = have ? 1.0f / l_sum : 0.0f;
+        const float lse_val = have ? (m_ref + log2f(l_sum)) * LN2 : -INFINITY;
+        const long long BH = static_cast<long long>(p.B) * p.H;
+#pragma unroll 1
+        for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t o[32];
+            if (have) {
+                tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            if (!in_range) continue;
+            if constexpr (SPLIT) {
+                float* dst = p.part_out + ((static_cast<long long>(split) * BH + bh) * p.Tq + row) * D + oc * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    float4 v4 = make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                                            __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+                    *reinterpret_cast<float4*>(dst + e) = v4;
+                }
+            } else {
+                __nv_bfloat16* dst = p.out + (static_cast<long long>(bh) * p.Tq + row) * D + oc * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 v4;
+                    v4.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+                    v4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+                    v4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+                    v4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+                    *reinterpret_cast<uint4*>(dst + e) = v4;
+                }
+            }
+        }
+        if (in_range) {
+            if constexpr (SPLIT) {
+                p.part_lse[(static_cast<long long>(split) * BH + bh) * p.Tq + row] = lse_val;
+            } else if (p.lse != nullptr) {
+                p.lse[static_cast<long long>(bh) * p.Tq + row] = lse_val;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+#undef BAR
+}
+
+// One warp per output row: lse = M + ln sum_c exp(lse_c - M), out = sum_c exp(lse_c - lse) O_c.
+template <int D>
+__global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_out,
+                                                          const float* __restrict__ part_lse, int C,
+                                                          long long rows, __nv_bfloat16* __restrict__ out,
+                                                          float* __restrict__ lse) {
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    float M = -INFINITY;
+    for (int c = lane; c < C; c += 32) M = fmaxf(M, __ldg(part_lse + c * rows + row));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    float L = -INFINITY;
+    if (M != -INFINITY) {
+        float s = 0.0f;
+        for (int c = lane; c < C; c += 32) s += expf(__ldg(part_lse + c * rows + row) - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        L = M + logf(s);
+        for (int c = 0; c < C; ++c) {
+            const float w = expf(__ldg(part_lse + c * rows + row) - L);
+            if (w == 0.0f) continue;   // an empty chunk (lse_c = -inf) adds nothing
+            const float* src = part_out + (static_cast<long long>(c) * rows + row) * D + lane * PER;
+            if constexpr (PER % 4 == 0) {
+#pragma unroll
+                for (int e = 0; e < PER; e += 4) {
+                    const float4 v4 = __ldg(reinterpret_cast<const float4*>(src + e));
+                    acc[e] += w * v4.x;
+                    acc[e + 1] += w * v4.y;
+                    acc[e + 2] += w * v4.z;
+                    acc[e + 3] += w * v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) acc[e] += w * __ldg(src + e);
+            }
+        }
+    }
+    __nv_bfloat16* dst = out + row * D + lane * PER;
+    if constexpr (PER == 1) {
+        dst[0] = __float2bfloat16_rn(acc[0]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < PER; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+    }
+    if (lane == 0 && lse != nullptr) lse[row] = L;
+}
+
+}  // namespace attn
+
+// =========================================================================== host side
+namespace {
+
+using attn::BM;
+using attn::BN;
+using attn::Cfg;
+using attn::Params;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+unsigned long long g_wait_ns = 1000000000ull;
+unsigned g_debug = 0;
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host checks that need no CUDA call.
+attn_status check_args(const void* q, const void* k, const void* v, const void* kv_len, const void* out,
+                       int B, int H, int Tq, int Tk, int D, float scale) {
+    if (!q || !k || !v || !kv_len || !out) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || Tq <= 0 || Tk <= 0) return ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (D != 32 && D != 64 && D != 256) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// Device must be compute capability 10.0 (B200 / sm_100a).  Cached per device ordinal.
+attn_status check_device() {
+    static int cached[64];
+    static std::once_flag once;
+    std::call_once(once, [] {
+        for (int i = 0; i < 64; ++i) cached[i] = -1;
+    });
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
+    if (cached[dev] < 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 0;
+    }
+    return cached[dev] ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
+// 3-D map over a [B*H, T, D] bf16 tensor; box = (swizzle block columns, rows, 1).
+bool make_map(CUtensorMap* map, const void* base, int T, long long BH, int D, int box_cols, int box_rows,
+              CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2ull, static_cast<cuuint64_t>(T) * D * 2ull};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, bool SPLIT>
+attn_status launch_fwd(const void* q, const void* k, const void* v, Params prm, cudaStream_t stream) {
+    using C = Cfg<D>;
+    const long long BH = static_cast<long long>(prm.B) * prm.H;
+    const CUtensorMapSwizzle swz = (C::SW == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, prm.Tq, BH, D, C::BLK, BM, swz) || !make_map(&mk, k, prm.Tk, BH, D, C::BLK, BN, swz) ||
+        !make_map(&mv, v, prm.Tk, BH, D, C::BLK, C::V_ROWS, swz))
+        return ATTN_ERR_CUDA;
+    const long long grid = static_cast<long long>(prm.n_qtiles) * BH * (SPLIT ? prm.num_splits : 1);
+    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    auto kern = attn::attn_fwd_kernel<D, SPLIT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    kern<<<static_cast<unsigned>(grid), attn::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+template <bool SPLIT>
+attn_status dispatch_fwd(int D, const void* q, const void* k, const void* v, const Params& prm,
+                         cudaStream_t stream) {
+    switch (D) {
+        case 32: return launch_fwd<32, SPLIT>(q, k, v, prm, stream);
+        case 64: return launch_fwd<64, SPLIT>(q, k, v, prm, stream);
+        case 256: return launch_fwd<256, SPLIT>(q, k, v, prm, stream);
+        default: return ATTN_ERR_UNSUPPORTED;
+    }
+}
+
+Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, float scale) {
+    Params prm;
+    memset(&prm, 0, sizeof prm);
+    prm.kv_len = kv_len;
+    prm.B = B;
+    prm.H = H;
+    prm.Tq = Tq;
+    prm.Tk = Tk;
+    prm.n_qtiles = (Tq + BM - 1) / BM;
+    prm.num_splits = 1;
+    prm.chunk_len = Tk;
+    prm.scale_log2 = scale * attn::LOG2E;
+    prm.wait_ns = g_wait_ns;
+    prm.debug = g_debug;
+    return prm;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_prefix_fwd(const void* q, const void* k, const void* v, const int32_t* kv_len, void* out,
+                            float* lse, int B, int H, int Tq, int Tk, int D, float scale, cudaStream_t stream) {
+    attn_status st = check_args(q, k, v, kv_len, out, B, H, Tq, Tk, D, scale);
+    if (st != ATTN_OK) return st;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_device()) != ATTN_OK) return st;
+    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    return dispatch_fwd<false>(D, q, k, v, prm, stream);
+}
+
+int attn_split_chunk_len(int Tk, int num_splits) {
+    if (Tk <= 0 || num_splits < 1 || num_splits > 1024) return 0;
+    long long per = (static_cast<long long>(Tk) + num_splits - 1) / num_splits;
+    per = (per + BN - 1) / BN * BN;
+    return static_cast<int>(per);
+}
+
+size_t attn_split_lse_offset(int num_splits, int B, int H, int Tq, int D) {
+    if (num_splits < 1 || B <= 0 || H <= 0 || Tq <= 0 || D <= 0) return 0;
+    size_t o = static_cast<size_t>(num_splits) * B * H * Tq * D * sizeof(float);
+    return (o + 255) / 256 * 256;
+}
+
+size_t attn_split_workspace_bytes(int num_splits, int B, int H, int Tq, int D) {
+    size_t off = attn_split_lse_offset(num_splits, B, H, Tq, D);
+    if (off == 0) return 0;
+    return off + static_cast<size_t>(num_splits) * B * H * Tq * sizeof(float);
+}
+
+attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                                  int num_splits, float* part_out, float* part_lse, int B, int H, int Tq, int Tk,
+                                  int D, float scale, cudaStream_t stream) {
+    attn_status st = check_args(q, k, v, kv_len, part_out, B, H, Tq, Tk, D, scale);
+    if (st != ATTN_OK) return st;
+    if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_device()) != ATTN_OK) return st;
+    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    prm.part_out = part_out;
+    prm.part_lse = part_lse;
+    prm.num_splits = num_splits;
+    prm.chunk_len = attn_split_chunk_len(Tk, num_splits);
+    return dispatch_fwd<true>(D, q, k, v, prm, stream);
+}
+
+attn_status attn_lse_combine(const float* part_out, const float* part_lse, int num_splits, void* out, float* lse,
+                             int B, int H, int Tq, int D, cudaStream_t stream) {
+    if (!part_out || !part_lse || !out) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(part_out) || !aligned16(out) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return ATTN_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > 1024 || B <= 0 || H <= 0 || Tq <= 0) return ATTN_ERR_INVALID_ARG;
+    if (D != 32 && D != 64 && D != 256) return ATTN_ERR_UNSUPPORTED;
+    attn_status st = check_device();
+    if (st != ATTN_OK) return st;
+    const long long rows = static_cast<long long>(B) * H * Tq;
+    const long long blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    switch (D) {
+        case 32: attn::lse_combine_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
+        case 64: attn::lse_combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
+        default: attn::lse_combine_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
+    }
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+attn_status attn_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    unsigned int flags = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&flags, attn::g_attn_status, sizeof flags) != cudaSuccess ||
+        cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (flags & attn::STATUS_TIMEOUT) return ATTN_ERR_TIMEOUT;
+    if (flags & attn::STATUS_KVLEN) return ATTN_ERR_KVLEN_RANGE;
+    return ATTN_OK;
+}
+
+void attn_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns < 1000000ull ? 1000000ull : ns; }
+
+void attn_set_debug_flags(unsigned flags) { g_debug = flags; }
+
+const char* attn_status_string(attn_status s) {
+    switch (s) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+        case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+        case ATTN_ERR_KVLEN_RANGE: return "ATTN_ERR_KVLEN_RANGE";
+    }
+    return "ATTN_ERR_UNKNOWN";
+}
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"
