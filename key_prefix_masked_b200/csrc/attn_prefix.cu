@@ -72,23 +72,27 @@ struct Cfg {
     static constexpr int VCH = NBLK;                  // V tile: chunks of V_ROWS key rows
     static constexpr int V_ROWS = BN / VCH;
     static constexpr int NSLOTS_RAW = (SMEM_LIMIT - Q_BYTES - 2048) / SLOT;
-    static constexpr int NSLOTS = NSLOTS_RAW > 16 ? 16 : NSLOTS_RAW;
+    static constexpr int GRP = (KCH >= 2) ? 2 : 1;      // chunks per ring group (one barrier pair)
+    static constexpr int NSLOTS_CAP = NSLOTS_RAW > 16 ? 16 : NSLOTS_RAW;
+    static constexpr int NSLOTS = NSLOTS_CAP / GRP * GRP;
+    static constexpr int NG = NSLOTS / GRP;             // ring groups
     static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOTS * SLOT + 1024;
     static constexpr uint32_t LAYOUT = (SW == 128) ? 2u : 4u;
     static_assert(D % BLK == 0, "head dim must be a multiple of the swizzle block");
     static_assert(V_ROWS % 16 == 0, "value chunks must hold whole 16-key MMA steps");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+    static_assert(KCH % GRP == 0 && VCH % GRP == 0 && NG <= 16, "ring grouping");
 };
 
 // Barrier slots inside the shared-memory control block.
 enum : int {
     BAR_Q = 0,
-    BAR_FULL = 1,       // [16] slot filled (TMA tx)
-    BAR_EMPTY = 17,     // [16] slot consumed (tcgen05.commit)
+    BAR_FULL = 1,       // [16] ring group filled (TMA tx)
+    BAR_EMPTY = 17,     // [16] ring group consumed (tcgen05.commit)
     BAR_S = 33,         // [2] S_j ready in TMEM buffer j&1
     BAR_P = 35,         // [2] P_j stored over S_j (128 softmax arrivals)
-    BAR_O = 37,         // [2] PV_j complete (buffer j&1)
+    BAR_O = 37,         // PV complete, announced for the last two tiles only
     BAR_DRAIN = 39,
     NUM_BARS = 40
 };
@@ -193,15 +197,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (tid == 0) {
         mbar_init(BAR(BAR_Q), 1);
-        for (int s = 0; s < 16; ++s) {
-            mbar_init(BAR(BAR_FULL + s), 1);
-            mbar_init(BAR(BAR_EMPTY + s), 1);
+        for (int g = 0; g < C::NG; ++g) {
+            mbar_init(BAR(BAR_FULL + g), 1);
+            mbar_init(BAR(BAR_EMPTY + g), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(BAR_S + i), 1);
             mbar_init(BAR(BAR_P + i), 128);
-            mbar_init(BAR(BAR_O + i), 1);
         }
+        mbar_init(BAR(BAR_O), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -218,6 +222,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 4) {
         // ================================================================ producer
+        // Loads go out in the order the MMA thread consumes them: K_0, K_1, then
+        // V_j, K_{j+2} for every tile j.  Each tile half is GRP-chunk groups; one ring
+        // group (GRP consecutive 16 KB slots) has one full and one empty barrier.
         if (lane == 0 && n_tiles > 0) {
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
@@ -227,49 +234,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int blk = 0; blk < C::NBLK; ++blk)
                 tma_load_3d(sQ_addr + blk * BM * C::SW, &tm_q, blk * C::BLK, q0, bh, BAR(BAR_Q));
 
-            int slot = 0;
+            int gi = 0;
             uint32_t phase = 0;
-            uint32_t pending = 0, pend_parity = 0;   // per-slot: fill issued, its parity
+            uint32_t pending = 0, pend_parity = 0;   // per ring group: fill issued, its parity
             int dropped = -1;
             bool ok = true;
-            auto next_slot = [&]() {
-                if (++slot == C::NSLOTS) {
-                    slot = 0;
+            auto acquire = [&]() -> bool {
+                ok = wait_bar(BAR(BAR_EMPTY + gi), phase ^ 1u, abort_flag, wlim);
+                if (ok) mbar_arrive_expect_tx(BAR(BAR_FULL + gi), C::GRP * C::SLOT);
+                return ok;
+            };
+            auto release_slot_bookkeeping = [&]() {
+                pending |= 1u << gi;
+                pend_parity = (pend_parity & ~(1u << gi)) | (phase << gi);
+                if (++gi == C::NG) {
+                    gi = 0;
                     phase ^= 1u;
                 }
             };
             auto load_k = [&](int j) {
                 const int key0 = k_begin + j * BN;
 #pragma unroll 1
-                for (int c = 0; c < C::KCH && ok; ++c) {
-                    ok = wait_bar(BAR(BAR_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(BAR(BAR_FULL + slot), C::SLOT);
-                    if ((p.debug & ATTN_DEBUG_DROP_COPY) && j == 0 && c == 0) {
-                        dropped = slot;   // announced but never issued: the consumer times out
-                    } else {
-                        tma_load_3d(sKV_addr + slot * C::SLOT, &tm_k, c * C::BLK, key0, bh,
-                                    BAR(BAR_FULL + slot));
-                        pending |= 1u << slot;
-                        pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
+                for (int g = 0; g < C::KCH / C::GRP && ok; ++g) {
+                    if (!acquire()) break;
+#pragma unroll
+                    for (int cc = 0; cc < C::GRP; ++cc) {
+                        const int c = g * C::GRP + cc;
+                        if ((p.debug & ATTN_DEBUG_DROP_COPY) && j == 0 && c == 0) {
+                            dropped = gi;   // announced, never issued: the consumer's wait runs out
+                            continue;
+                        }
+                        tma_load_3d(sKV_addr + (gi * C::GRP + cc) * C::SLOT, &tm_k, c * C::BLK, key0, bh,
+                                    BAR(BAR_FULL + gi));
                     }
-                    next_slot();
+                    release_slot_bookkeeping();
                 }
             };
             auto load_v = [&](int j) {
                 const int key0 = k_begin + j * BN;
 #pragma unroll 1
-                for (int c = 0; c < C::VCH && ok; ++c) {
-                    ok = wait_bar(BAR(BAR_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(BAR(BAR_FULL + slot), C::SLOT);
+                for (int g = 0; g < C::VCH / C::GRP && ok; ++g) {
+                    if (!acquire()) break;
 #pragma unroll
-                    for (int blk = 0; blk < C::NBLK; ++blk)
-                        tma_load_3d(sKV_addr + slot * C::SLOT + blk * C::V_ROWS * C::SW, &tm_v,
-                                    blk * C::BLK, key0 + c * C::V_ROWS, bh, BAR(BAR_FULL + slot));
-                    pending |= 1u << slot;
-                    pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
-                    next_slot();
+                    for (int cc = 0; cc < C::GRP; ++cc) {
+                        const int c = g * C::GRP + cc;
+#pragma unroll
+                        for (int blk = 0; blk < C::NBLK; ++blk)
+                            tma_load_3d(sKV_addr + (gi * C::GRP + cc) * C::SLOT + blk * C::V_ROWS * C::SW, &tm_v,
+                                        blk * C::BLK, key0 + c * C::V_ROWS, bh, BAR(BAR_FULL + gi));
+                    }
+                    release_slot_bookkeeping();
                 }
             };
             load_k(0);
@@ -282,101 +296,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!ok) {
                 // Drain: every copy issued must land before this CTA's memory is reused.
                 wait_bar_drain(BAR(BAR_Q), 0, wlim);
-                for (int s = 0; s < C::NSLOTS; ++s)
-                    if (((pending >> s) & 1u) && s != dropped)
-                        wait_bar_drain(BAR(BAR_FULL + s), (pend_parity >> s) & 1u, wlim);
+                for (int g = 0; g < C::NG; ++g)
+                    if (((pending >> g) & 1u) && g != dropped)
+                        wait_bar_drain(BAR(BAR_FULL + g), (pend_parity >> g) & 1u, wlim);
             }
         }
         __syncwarp();
     } else if (warp == 5) {
-        // ================================================================ MMA issuer
-        if (n_tiles > 0) {
+        // ================================================================ MMA issuer (one thread)
+        if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(BM, BN, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(BM, D, true);
-            int slot = 0;
+            // Descriptor templates; the 14-bit address field is advanced by plain adds.
+            const uint64_t q_desc0 = make_smem_desc(sQ_addr, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t k_desc0 = make_smem_desc(sKV_addr, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
+            int gi = 0;
             uint32_t phase = 0;
             bool ok = wait_bar(BAR(BAR_Q), 0, abort_flag, wlim);
-            ok = __all_sync(0xffffffffu, ok);
-            auto next_slot = [&]() {
-                if (++slot == C::NSLOTS) {
-                    slot = 0;
+            auto next_group = [&]() {
+                if (++gi == C::NG) {
+                    gi = 0;
                     phase ^= 1u;
                 }
             };
             auto issue_s = [&](int j) {
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
 #pragma unroll 1
-                for (int c = 0; c < C::KCH; ++c) {
-                    ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_FULL + slot), phase, abort_flag, wlim));
+                for (int g = 0; g < C::KCH / C::GRP; ++g) {
+                    ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
                     if (!ok) return;
                     tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t a_base = sQ_addr + c * BM * C::SW;
-                        const uint32_t b_base = sKV_addr + slot * C::SLOT;
 #pragma unroll
-                        for (int kk = 0; kk < C::BLK / 16; ++kk) {
-                            const uint64_t ad = make_smem_desc(a_base + kk * 32, 16, 8 * C::SW, C::LAYOUT);
-                            const uint64_t bd = make_smem_desc(b_base + kk * 32, 16, 8 * C::SW, C::LAYOUT);
-                            mma_ss(d_tmem, ad, bd, IDESC_S, (c | kk) != 0 ? 1u : 0u);
-                        }
-                        tc_commit(BAR(BAR_EMPTY + slot));
+                    for (int cc = 0; cc < C::GRP; ++cc) {
+                        const int c = g * C::GRP + cc;
+                        const uint64_t ad = q_desc0 + static_cast<uint64_t>((c * BM * C::SW) >> 4);
+                        const uint64_t bd = k_desc0 + static_cast<uint64_t>(((gi * C::GRP + cc) * C::SLOT) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < C::BLK / 16; ++kk)
+                            mma_ss(d_tmem, ad + static_cast<uint64_t>(kk * 2), bd + static_cast<uint64_t>(kk * 2),
+                                   IDESC_S, (c | kk) != 0 ? 1u : 0u);
                     }
-                    __syncwarp();
-                    next_slot();
+                    tc_commit(BAR(BAR_EMPTY + gi));
+                    next_group();
                 }
-                if (lane == 0) tc_commit(BAR(BAR_S + (j & 1)));
-                __syncwarp();
+                tc_commit(BAR(BAR_S + (j & 1)));
             };
             auto issue_pv = [&](int j) {
-                ok = __all_sync(0xffffffffu,
-                                wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
                 if (!ok) return;
                 tc_fence_after();
                 const int valid = min(BN, k_end - (k_begin + j * BN));
                 const int kblocks = (valid + 15) >> 4;   // 16-key steps holding a valid key
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
 #pragma unroll 1
-                for (int c = 0; c < C::VCH; ++c) {
-                    ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_FULL + slot), phase, abort_flag, wlim));
+                for (int g = 0; g < C::VCH / C::GRP; ++g) {
+                    ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
                     if (!ok) return;
                     tc_fence_after();
-                    const uint32_t v_base = sKV_addr + slot * C::SLOT;
-                    // Zero value rows in [valid, 16*kblocks) that fall inside this chunk.
-                    const int r0 = max(valid, c * C::V_ROWS);
-                    const int r1 = min(kblocks * 16, (c + 1) * C::V_ROWS);
-                    if (r1 > r0) {
-                        constexpr int PIECES = C::SW / 16;   // 16-byte pieces per row segment
-                        const int total = (r1 - r0) * C::NBLK * PIECES;
-                        uint8_t* vs = sKV + slot * C::SLOT;
-                        for (int i = lane; i < total; i += 32) {
-                            const int piece = i % PIECES;
-                            const int rb = i / PIECES;
-                            const int blk = rb % C::NBLK;
-                            const int r = r0 + rb / C::NBLK - c * C::V_ROWS;
-                            *reinterpret_cast<uint4*>(vs + blk * C::V_ROWS * C::SW + r * C::SW + piece * 16) =
-                                make_uint4(0u, 0u, 0u, 0u);
+                    if (valid < BN) {
+                        // Zero value rows in [valid, 16*kblocks) held by this group's chunks.
+                        bool wrote = false;
+                        for (int cc = 0; cc < C::GRP; ++cc) {
+                            const int c = g * C::GRP + cc;
+                            const int r0 = max(valid, c * C::V_ROWS);
+                            const int r1 = min(kblocks * 16, (c + 1) * C::V_ROWS);
+                            uint8_t* vs = sKV + (gi * C::GRP + cc) * C::SLOT;
+                            for (int r = r0; r < r1; ++r)
+                                for (int blk = 0; blk < C::NBLK; ++blk)
+                                    for (int piece = 0; piece < C::SW / 16; ++piece) {
+                                        *reinterpret_cast<uint4*>(vs + blk * C::V_ROWS * C::SW +
+                                                                  (r - c * C::V_ROWS) * C::SW + piece * 16) =
+                                            make_uint4(0u, 0u, 0u, 0u);
+                                        wrote = true;
+                                    }
                         }
-                        fence_proxy_async_smem();
-                        __syncwarp();
+                        if (wrote) fence_proxy_async_smem();
                     }
-                    if (lane == 0) {
+#pragma unroll
+                    for (int cc = 0; cc < C::GRP; ++cc) {
+                        const int c = g * C::GRP + cc;
+                        const uint64_t bd = v_desc0 + static_cast<uint64_t>(((gi * C::GRP + cc) * C::SLOT) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
                             const int kb = c * (C::V_ROWS / 16) + kk;
-                            if (kb < kblocks) {
-                                const uint64_t bd = make_smem_desc(v_base + kk * 16 * C::SW,
-                                                                   C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
-                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u, bd, IDESC_PV,
+                            if (kb < kblocks)
+                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                       bd + static_cast<uint64_t>((kk * 16 * C::SW) >> 4), IDESC_PV,
                                        (j == 0 && kb == 0) ? 0u : 1u);
-                            }
                         }
-                        tc_commit(BAR(BAR_EMPTY + slot));
                     }
-                    __syncwarp();
-                    next_slot();
+                    tc_commit(BAR(BAR_EMPTY + gi));
+                    next_group();
                 }
-                if (lane == 0) tc_commit(BAR(BAR_O + (j & 1)));
-                __syncwarp();
+                // O is announced only after the last two PV steps: the softmax rescale of
+                // the last tile and the epilogue are its only readers (earlier rescales
+                // learn that PV_{j-1} is done from S_{j+1}, issued after it).
+                if (j >= n_tiles - 2) tc_commit(BAR(BAR_O));
             };
             if (ok) issue_s(0);
             if (ok && n_tiles > 1) issue_s(1);
@@ -386,8 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (ok && j + 2 < n_tiles) issue_s(j + 2);
             }
             // Drain: every MMA issued completes before TMEM is released.
-            if (lane == 0) tc_commit(BAR(BAR_DRAIN));
-            __syncwarp();
+            tc_commit(BAR(BAR_DRAIN));
             wait_bar_drain(BAR(BAR_DRAIN), 0, wlim);
         }
         __syncwarp();
@@ -395,6 +410,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // ================================================================ softmax
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const float sl2 = p.scale_log2;
+        const bool pos_scale = sl2 > 0.0f;
         float m_ref = -INFINITY;   // reference max, log2 domain
         float l_sum = 0.0f;        // row sum relative to m_ref
         bool ok = true;
@@ -408,20 +424,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld128_wait(s_addr, raw);
             float x[BN];
             const int valid = min(BN, k_end - (k_begin + j * BN));
-            float mx = -INFINITY;
-            if (valid >= BN) {
+            if (valid < BN) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    x[c] = __uint_as_float(raw[c]) * sl2;
-                    mx = fmaxf(mx, x[c]);
-                }
+                for (int c = 0; c < BN; ++c) x[c] = (c < valid) ? __uint_as_float(raw[c]) : -INFINITY;
             } else {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    x[c] = (c < valid) ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
-                    mx = fmaxf(mx, x[c]);
-                }
+                for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(raw[c]);
             }
+            if (!pos_scale) {
+                // zero or negative scale: scale every finite score first (the max flips)
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = (c < valid) ? x[c] * sl2 : -INFINITY;
+            }
+            // tree max over the row
+            float mxp[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) mxp[t] = x[t];
+#pragma unroll
+            for (int c = 8; c < BN; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) *
+                             (pos_scale ? sl2 : 1.0f);
             float factor = 1.0f;
             bool rescale = false;
             if (j == 0) {
@@ -432,24 +455,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 m_ref = m_new;
                 rescale = true;
             }
-            float tile_sum = 0.0f;
+            const float mul = pos_scale ? sl2 : 1.0f;
+            const float neg_m = -m_ref;
+            float sp[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(x[cc * 32 + 2 * e] - m_ref);
-                    const float p1 = fast_exp2(x[cc * 32 + 2 * e + 1] - m_ref);
-                    tile_sum += p0 + p1;
+                    const float p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
+                    const float p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
+                    sp[e & 7] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(s_addr + cc * 16, pk);
             }
+            const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l_sum = l_sum * factor + tile_sum;
             if (rescale) {
-                // O may only be touched once PV_{j-1} has completed.
-                ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_O + ((j - 1) & 1)), ((j - 1) >> 1) & 1,
-                                                      abort_flag, wlim));
+                // O may only be touched once PV_{j-1} has completed: S_{j+1} was issued
+                // after it, and for the last tile the MMA thread announces PV_{n-2}.
+                const bool w = (j + 1 < n_tiles)
+                                   ? wait_bar(BAR(BAR_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
+                                   : wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
+                ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll 1
@@ -465,10 +496,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_before();
             mbar_arrive(BAR(BAR_P + (j & 1)));
         }
-        // ---- epilogue
+        // ---- epilogue: the O barrier completes once per PV among the last two
         if (ok && n_tiles > 0) {
-            const int jl = n_tiles - 1;
-            ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_O + (jl & 1)), (jl >> 1) & 1, abort_flag, wlim));
+            bool w = wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
+            if (n_tiles > 1) w = w && wait_bar(BAR(BAR_O), 1, abort_flag, wlim);
+            ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }
         const int row = q0 + tid;

@@ -55,6 +55,9 @@ WORKLOADS = {
                        ragged_seed_draw=True),
     "splitkv": Workload("splitkv", 1, 8, 256, 1024, 1000000, (1000000,), 0.5, False,
                         num_splits=64),
+    # a reduced icl shape for profiler captures: same head dim, padding and value
+    # distribution, inputs (161 MB) still larger than the L2
+    "icl_profile": Workload("icl_profile", 1, 8, 256, 8192, 16512, (16384,), 0.5, True),
 }
 
 
