@@ -95,6 +95,33 @@ attn_status attn_lse_combine(const float* part_out, const float* part_lse, int n
                              void* out, float* lse, int B, int H, int Tq, int D,
                              cudaStream_t stream);
 
+/* Split-KV forward that allocates nothing, for callers that cannot call cudaMalloc.
+ * The pages have no counterpart to this entry point: it exists for the integration
+ * side, not for the method.  Some callers only ever receive device memory for their
+ * inputs and outputs: a hook running inside another framework whose allocator owns all
+ * of device memory, a runtime that fixes its memory plan at start-up, or a real-time
+ * loop that cannot take the device-wide synchronisation a cudaMalloc may imply.  For
+ * them the split partials live in one file-scope device array of the library
+ * (ATTN_NOALLOC_SCRATCH_BYTES = 64 MiB), which every GPU that loads the library holds
+ * until the process exits.
+ *   Same arguments and result as attn_prefix_fwd_split followed by attn_lse_combine:
+ *   out bf16 [B,H,Tq,D], lse fp32 [B,H,Tq] or NULL.
+ *   Shapes whose split workspace, attn_split_workspace_bytes(num_splits, B, H, Tq, D),
+ *   exceeds ATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_INVALID_ARG before any
+ *   CUDA call.
+ *   The first call on a device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   Every call shares the one array and leaves its partials there; each call writes
+ *   every partial it reads, so nothing needs clearing, but calls whose work overlaps on
+ *   the GPU (other streams, other host threads) race on the array and must be serialised
+ *   by the caller. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+attn_status attn_prefix_fwd_splitkv_noalloc(const void* q, const void* k, const void* v,
+                                            const int32_t* kv_len, int num_splits,
+                                            void* out, float* lse,
+                                            int B, int H, int Tq, int Tk, int D, float scale,
+                                            cudaStream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the sticky device flags raised by
  * earlier launches: ATTN_ERR_TIMEOUT has priority over ATTN_ERR_KVLEN_RANGE; ATTN_OK if
  * none.  A CUDA error during the synchronization returns ATTN_ERR_CUDA. */

@@ -37,6 +37,7 @@ _SIGNATURES = {
     "attn_split_lse_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_prefix_fwd_split": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_lse_combine": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_prefix_fwd_splitkv_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "attn_set_debug_flags": (None, [ctypes.c_uint]),

@@ -854,3 +854,54 @@ const char* attn_status_string(attn_status s) {
 int attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation split-KV
+// The partials of attn_prefix_fwd_splitkv_noalloc live here instead of in caller memory.
+// In host code this name is only a host-side stand-in for the array: its device address
+// comes from cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (nullptr on failure).
+void* noalloc_scratch_on_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" attn_status attn_prefix_fwd_splitkv_noalloc(const void* q, const void* k, const void* v,
+                                                       const int32_t* kv_len, int num_splits, void* out, float* lse,
+                                                       int B, int H, int Tq, int Tk, int D, float scale,
+                                                       cudaStream_t stream) {
+    attn_status st = check_args(q, k, v, kv_len, out, B, H, Tq, Tk, D, scale);
+    if (st != ATTN_OK) return st;
+    if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_split_workspace_bytes(num_splits, B, H, Tq, D);
+    if (need == 0 || need > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES)) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_device()) != ATTN_OK) return st;
+    unsigned char* scratch = static_cast<unsigned char*>(noalloc_scratch_on_current_device());
+    if (scratch == nullptr) return ATTN_ERR_CUDA;
+    float* part_out = reinterpret_cast<float*>(scratch);
+    float* part_lse = reinterpret_cast<float*>(scratch + attn_split_lse_offset(num_splits, B, H, Tq, D));
+    st = attn_prefix_fwd_split(q, k, v, kv_len, num_splits, part_out, part_lse, B, H, Tq, Tk, D, scale, stream);
+    if (st != ATTN_OK) return st;
+    return attn_lse_combine(part_out, part_lse, num_splits, out, lse, B, H, Tq, D, stream);
+}
