@@ -50,7 +50,7 @@ namespace attn {
 
 constexpr int BM = 128;               // query rows per CTA (one TMEM lane each)
 constexpr int BN = 128;               // keys per tile
-constexpr int NUM_THREADS = 192;      // 4 softmax warps + producer warp + MMA warp
+constexpr int NUM_THREADS = 224;      // 4 softmax warps + producer + MMA issuer + wait relay
 constexpr int SMEM_LIMIT = 232448;    // 227 KB opt-in dynamic shared memory per block
 constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128) S1 [128,256) O [256, 256+D)
 constexpr uint32_t O_COL = 256;
@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::NSLOTS * C::SLOT);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    uint32_t* ready_seq = tmem_holder + 2;   // events the relay warp has seen complete
+    const uint32_t ready_addr = smem_u32(ready_seq);
     const uint32_t bar0 = smem_u32(bars);
     const uint32_t sQ_addr = smem_u32(sQ);
     const uint32_t sKV_addr = smem_u32(sKV);
@@ -208,6 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(BAR(BAR_O), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
         *abort_flag = 0;
+        *ready_seq = 0u;
         fence_mbar_init();
     }
     if (warp == 5) {
@@ -313,6 +316,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
             int gi = 0;
             uint32_t phase = 0;
+            uint32_t consumed = 0;
             bool ok = wait_bar(BAR(BAR_Q), 0, abort_flag, wlim);
             auto next_group = [&]() {
                 if (++gi == C::NG) {
@@ -320,11 +324,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     phase ^= 1u;
                 }
             };
+            // The relay warp performs the blocking mbarrier waits in this thread's order
+            // and publishes how many events have completed; polling that word costs a
+            // shared-memory load instead of an mbarrier round trip.
+            auto next_event = [&]() -> bool {
+                ++consumed;
+                if (ld_acquire_smem(ready_addr) >= consumed) return true;
+                const uint64_t t0 = global_timer_ns();
+                while (true) {
+                    if (ld_acquire_smem(ready_addr) >= consumed) return true;
+                    if (*abort_flag) return false;
+                    if (global_timer_ns() - t0 > wlim) {
+                        *abort_flag = 1;
+                        atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                        return false;
+                    }
+                }
+            };
             auto issue_s = [&](int j) {
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
 #pragma unroll 1
                 for (int g = 0; g < C::KCH / C::GRP; ++g) {
-                    ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
+                    ok = next_event();
                     if (!ok) return;
                     tc_fence_after();
 #pragma unroll
@@ -343,7 +364,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_commit(BAR(BAR_S + (j & 1)));
             };
             auto issue_pv = [&](int j) {
-                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                ok = next_event();   // P_j stored
                 if (!ok) return;
                 tc_fence_after();
                 const int valid = min(BN, k_end - (k_begin + j * BN));
@@ -351,9 +372,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
 #pragma unroll 1
                 for (int g = 0; g < C::VCH / C::GRP; ++g) {
-                    ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
+                    ok = next_event();
                     if (!ok) return;
                     tc_fence_after();
+                    (void)phase;
                     if (valid < BN) {
                         // Zero value rows in [valid, 16*kblocks) held by this group's chunks.
                         bool wrote = false;
@@ -404,6 +426,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // Drain: every MMA issued completes before TMEM is released.
             tc_commit(BAR(BAR_DRAIN));
             wait_bar_drain(BAR(BAR_DRAIN), 0, wlim);
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // ================================================================ wait relay
+        // Waits on every ring group and P barrier in the MMA thread's consumption order
+        // (S_0, S_1, then P_j, V_j, S_{j+2}) and publishes the count of completed events
+        // with a release store; the MMA thread acquires it.
+        if (lane == 0 && n_tiles > 0) {
+            int gi = 0;
+            uint32_t phase = 0, seq = 0;
+            bool ok = true;
+            auto group = [&]() {
+                ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
+                if (!ok) return;
+                st_release_smem(ready_addr, ++seq);
+                if (++gi == C::NG) {
+                    gi = 0;
+                    phase ^= 1u;
+                }
+            };
+            auto relay_s = [&](int) {
+                for (int g = 0; g < C::KCH / C::GRP && ok; ++g) group();
+            };
+            auto relay_pv = [&](int j) {
+                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                if (!ok) return;
+                st_release_smem(ready_addr, ++seq);
+                for (int g = 0; g < C::VCH / C::GRP && ok; ++g) group();
+            };
+            relay_s(0);
+            if (ok && n_tiles > 1) relay_s(1);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                relay_pv(j);
+                if (ok && j + 2 < n_tiles) relay_s(j + 2);
+            }
         }
         __syncwarp();
     } else {
