@@ -307,23 +307,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else if (warp == 5) {
         // ================================================================ MMA issuer (one thread)
+        // Two readiness events per tile, published by the relay warp: "P_j stored and
+        // V_j landed" and "K_{j+2} landed".  Between them the 8 PV and 16 S MMAs of a
+        // tile are issued as straight-line code from precomputed descriptors, so the
+        // tensor pipe's queue stays fed (the tile's MMA mix alone runs at the tensor
+        // peak; the issuing thread's overhead is what decides the rate).
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(BM, BN, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(BM, D, true);
+            constexpr int KG = C::KCH / C::GRP;
+            constexpr int VG = C::VCH / C::GRP;
+            constexpr uint32_t GSTEP = static_cast<uint32_t>((C::GRP * C::SLOT) >> 4);   // per ring group
             // Descriptor templates; the 14-bit address field is advanced by plain adds.
             const uint64_t q_desc0 = make_smem_desc(sQ_addr, 16, 8 * C::SW, C::LAYOUT);
             const uint64_t k_desc0 = make_smem_desc(sKV_addr, 16, 8 * C::SW, C::LAYOUT);
             const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
-            int gi = 0;
-            uint32_t phase = 0;
+            int gi = 0;   // ring group of the next K/V group to consume
             uint32_t consumed = 0;
             bool ok = wait_bar(BAR(BAR_Q), 0, abort_flag, wlim);
-            auto next_group = [&]() {
-                if (++gi == C::NG) {
-                    gi = 0;
-                    phase ^= 1u;
-                }
-            };
+            auto ring = [&](int g) { return (gi + g < C::NG) ? gi + g : gi + g - C::NG; };
+            auto advance = [&](int n) { gi = (gi + n < C::NG) ? gi + n : gi + n - C::NG; };
             // The relay warp performs the blocking mbarrier waits in this thread's order
             // and publishes how many events have completed; polling that word costs a
             // shared-memory load instead of an mbarrier round trip.
@@ -343,47 +346,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             };
             auto issue_s = [&](int j) {
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
-#pragma unroll 1
-                for (int g = 0; g < C::KCH / C::GRP; ++g) {
-                    ok = next_event();
-                    if (!ok) return;
-                    tc_fence_after();
+#pragma unroll
+                for (int g = 0; g < KG; ++g) {
+                    const uint64_t kd = k_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
 #pragma unroll
                     for (int cc = 0; cc < C::GRP; ++cc) {
                         const int c = g * C::GRP + cc;
-                        const uint64_t ad = q_desc0 + static_cast<uint64_t>((c * BM * C::SW) >> 4);
-                        const uint64_t bd = k_desc0 + static_cast<uint64_t>(((gi * C::GRP + cc) * C::SLOT) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < C::BLK / 16; ++kk)
-                            mma_ss(d_tmem, ad + static_cast<uint64_t>(kk * 2), bd + static_cast<uint64_t>(kk * 2),
-                                   IDESC_S, (c | kk) != 0 ? 1u : 0u);
+                            mma_ss(d_tmem, q_desc0 + static_cast<uint64_t>(((c * BM * C::SW) >> 4) + kk * 2),
+                                   kd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + kk * 2), IDESC_S,
+                                   (c | kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit(BAR(BAR_EMPTY + gi));
-                    next_group();
                 }
+#pragma unroll
+                for (int g = 0; g < KG; ++g) tc_commit(BAR(BAR_EMPTY + ring(g)));
                 tc_commit(BAR(BAR_S + (j & 1)));
+                advance(KG);
             };
             auto issue_pv = [&](int j) {
-                ok = next_event();   // P_j stored
-                if (!ok) return;
-                tc_fence_after();
                 const int valid = min(BN, k_end - (k_begin + j * BN));
-                const int kblocks = (valid + 15) >> 4;   // 16-key steps holding a valid key
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
-#pragma unroll 1
-                for (int g = 0; g < C::VCH / C::GRP; ++g) {
-                    ok = next_event();
-                    if (!ok) return;
-                    tc_fence_after();
-                    (void)phase;
-                    if (valid < BN) {
-                        // Zero value rows in [valid, 16*kblocks) held by this group's chunks.
-                        bool wrote = false;
+                if (valid == BN) {
+                    const uint32_t acc0 = (j == 0) ? 0u : 1u;
+#pragma unroll
+                    for (int g = 0; g < VG; ++g) {
+                        const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
+#pragma unroll
+                        for (int cc = 0; cc < C::GRP; ++cc) {
+#pragma unroll
+                            for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
+                                const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
+                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                       vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
+                                       IDESC_PV, kb == 0 ? acc0 : 1u);
+                            }
+                        }
+                    }
+                } else {
+                    // Partial tile: zero the value rows in [valid, 16*kblocks) and skip the
+                    // 16-key steps that hold no valid key.
+                    const int kblocks = (valid + 15) >> 4;
+                    bool wrote = false;
+                    for (int g = 0; g < VG; ++g) {
                         for (int cc = 0; cc < C::GRP; ++cc) {
                             const int c = g * C::GRP + cc;
                             const int r0 = max(valid, c * C::V_ROWS);
                             const int r1 = min(kblocks * 16, (c + 1) * C::V_ROWS);
-                            uint8_t* vs = sKV + (gi * C::GRP + cc) * C::SLOT;
+                            uint8_t* vs = sKV + (ring(g) * C::GRP + cc) * C::SLOT;
                             for (int r = r0; r < r1; ++r)
                                 for (int blk = 0; blk < C::NBLK; ++blk)
                                     for (int piece = 0; piece < C::SW / 16; ++piece) {
@@ -393,35 +403,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                         wrote = true;
                                     }
                         }
-                        if (wrote) fence_proxy_async_smem();
                     }
-#pragma unroll
-                    for (int cc = 0; cc < C::GRP; ++cc) {
-                        const int c = g * C::GRP + cc;
-                        const uint64_t bd = v_desc0 + static_cast<uint64_t>(((gi * C::GRP + cc) * C::SLOT) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
-                            const int kb = c * (C::V_ROWS / 16) + kk;
-                            if (kb < kblocks)
-                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                       bd + static_cast<uint64_t>((kk * 16 * C::SW) >> 4), IDESC_PV,
-                                       (j == 0 && kb == 0) ? 0u : 1u);
+                    if (wrote) fence_proxy_async_smem();
+                    for (int g = 0; g < VG; ++g) {
+                        const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
+                        for (int cc = 0; cc < C::GRP; ++cc) {
+                            for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
+                                const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
+                                if (kb < kblocks)
+                                    mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                           vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
+                                           IDESC_PV, (j == 0 && kb == 0) ? 0u : 1u);
+                            }
                         }
                     }
-                    tc_commit(BAR(BAR_EMPTY + gi));
-                    next_group();
                 }
+#pragma unroll
+                for (int g = 0; g < VG; ++g) tc_commit(BAR(BAR_EMPTY + ring(g)));
                 // O is announced only after the last two PV steps: the softmax rescale of
                 // the last tile and the epilogue are its only readers (earlier rescales
                 // learn that PV_{j-1} is done from S_{j+1}, issued after it).
                 if (j >= n_tiles - 2) tc_commit(BAR(BAR_O));
+                advance(VG);
             };
-            if (ok) issue_s(0);
-            if (ok && n_tiles > 1) issue_s(1);
+            if (ok) ok = next_event();
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+            }
+            if (ok && n_tiles > 1) {
+                ok = next_event();
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(1);
+                }
+            }
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
+                ok = next_event();   // P_j stored and V_j landed
+                if (!ok) break;
+                tc_fence_after();
                 issue_pv(j);
-                if (ok && j + 2 < n_tiles) issue_s(j + 2);
+                if (j + 2 < n_tiles) {
+                    ok = next_event();   // K_{j+2} landed
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(j + 2);
+                }
             }
             // Drain: every MMA issued completes before TMEM is released.
             tc_commit(BAR(BAR_DRAIN));
@@ -430,37 +458,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else if (warp == 6) {
         // ================================================================ wait relay
-        // Waits on every ring group and P barrier in the MMA thread's consumption order
-        // (S_0, S_1, then P_j, V_j, S_{j+2}) and publishes the count of completed events
-        // with a release store; the MMA thread acquires it.
+        // Waits on the ring groups and P barriers in the MMA thread's consumption order
+        // and publishes one completed event per MMA batch with a release store: K_0,
+        // K_1, then per tile j "P_j + V_j" and "K_{j+2}"; the MMA thread acquires it.
         if (lane == 0 && n_tiles > 0) {
             int gi = 0;
             uint32_t phase = 0, seq = 0;
             bool ok = true;
             auto group = [&]() {
-                ok = wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
-                if (!ok) return;
-                st_release_smem(ready_addr, ++seq);
+                ok = ok && wait_bar(BAR(BAR_FULL + gi), phase, abort_flag, wlim);
                 if (++gi == C::NG) {
                     gi = 0;
                     phase ^= 1u;
                 }
             };
-            auto relay_s = [&](int) {
-                for (int g = 0; g < C::KCH / C::GRP && ok; ++g) group();
+            auto publish = [&]() {
+                if (ok) st_release_smem(ready_addr, ++seq);
             };
-            auto relay_pv = [&](int j) {
-                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
-                if (!ok) return;
-                st_release_smem(ready_addr, ++seq);
-                for (int g = 0; g < C::VCH / C::GRP && ok; ++g) group();
+            auto relay_s = [&]() {
+                for (int g = 0; g < C::KCH / C::GRP; ++g) group();
+                publish();
             };
-            relay_s(0);
-            if (ok && n_tiles > 1) relay_s(1);
+            relay_s();
+            if (n_tiles > 1) relay_s();
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
-                relay_pv(j);
-                if (ok && j + 2 < n_tiles) relay_s(j + 2);
+                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                for (int g = 0; g < C::VCH / C::GRP; ++g) group();
+                publish();
+                if (j + 2 < n_tiles) relay_s();
             }
         }
         __syncwarp();
