@@ -60,6 +60,7 @@ constexpr float LOG2E = 1.44269504088896340736f;
 
 constexpr unsigned STATUS_TIMEOUT = 1u;
 constexpr unsigned STATUS_KVLEN = 2u;
+constexpr unsigned STATUS_LAYOUT = 4u;   // dynamic shared memory not 1024-byte aligned
 
 template <int D>
 struct Cfg {
@@ -147,6 +148,32 @@ __device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity,
                                             unsigned long long limit_ns) {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicOr(&g_attn_status, STATUS_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Cluster-scope variants for barriers completed by the other CTA of a pair.
+__device__ __noinline__ bool wait_bar_cl(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned long long limit_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicOr(&g_attn_status, STATUS_TIMEOUT);
+            return false;
+        }
+    }
+}
+__device__ __noinline__ bool wait_bar_drain_cl(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_cluster(bar, parity)) {
         if (global_timer_ns() - t0 > limit_ns) {
             atomicOr(&g_attn_status, STATUS_TIMEOUT);
             return false;
@@ -642,6 +669,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #undef BAR
 }
 
+#include "pair_kernel.cuh"
+
 // One warp per output row: lse = M + ln sum_c exp(lse_c - M), out = sum_c exp(lse_c - lse) O_c.
 template <int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_out,
@@ -801,13 +830,38 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, Params prm, 
     return ATTN_OK;
 }
 
+// Head dim 256 runs on CTA pairs: 256-row query tiles, each CTA copying half of K and V.
+template <bool SPLIT>
+attn_status launch_fwd_pair(const void* q, const void* k, const void* v, Params prm, cudaStream_t stream) {
+    using C = attn::PairCfg;
+    const long long BH = static_cast<long long>(prm.B) * prm.H;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, prm.Tq, BH, C::D, 64, C::ROWS, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, prm.Tk, BH, C::D, 64, C::KH, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, prm.Tk, BH, C::D, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return ATTN_ERR_CUDA;
+    prm.n_qtiles = (prm.Tq + 2 * C::ROWS - 1) / (2 * C::ROWS);
+    const long long grid = 2LL * prm.n_qtiles * BH * (SPLIT ? prm.num_splits : 1);
+    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    auto kern = attn::attn_fwd_pair_kernel<SPLIT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
 template <bool SPLIT>
 attn_status dispatch_fwd(int D, const void* q, const void* k, const void* v, const Params& prm,
                          cudaStream_t stream) {
     switch (D) {
         case 32: return launch_fwd<32, SPLIT>(q, k, v, prm, stream);
         case 64: return launch_fwd<64, SPLIT>(q, k, v, prm, stream);
-        case 256: return launch_fwd<256, SPLIT>(q, k, v, prm, stream);
+        case 256:
+            if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<256, SPLIT>(q, k, v, prm, stream);
+            return launch_fwd_pair<SPLIT>(q, k, v, prm, stream);
         default: return ATTN_ERR_UNSUPPORTED;
     }
 }
@@ -916,6 +970,7 @@ attn_status attn_get_device_status(cudaStream_t stream) {
     }
     if (flags & attn::STATUS_TIMEOUT) return ATTN_ERR_TIMEOUT;
     if (flags & attn::STATUS_KVLEN) return ATTN_ERR_KVLEN_RANGE;
+    if (flags & attn::STATUS_LAYOUT) return ATTN_ERR_CUDA;
     return ATTN_OK;
 }
 

@@ -1,0 +1,444 @@
+// pair_kernel.cuh -- head-dim-256 forward on a CTA pair (cta_group::2).  Included by
+// attn_prefix.cu inside namespace attn, after the single-CTA kernel's helpers.
+//
+// A cluster of two CTAs shares one 256-row query tile: each CTA holds its own 128 query
+// rows (Q in its shared memory, S / P / O in its TMEM lanes) and HALF of every key and
+// value tile -- keys [64r, 64r + 64) of K, value columns [128r, 128r + 128) of V for
+// CTA rank r.  The leader CTA's single MMA thread issues M = 256 tcgen05 MMAs that read
+// A from each CTA and B split across both, so each CTA streams 64 KB of K/V per 128-key
+// tile instead of 128 KB: the five 32 KB ring slots hold 2.5 tiles of look-ahead, which
+// takes the copy latency off the critical path.
+//
+// Roles (256 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
+// producer (both CTAs, into their own memory, completing on the leader's barriers);
+// warp 5 TMEM allocation (both) and MMA issue (leader); warp 6 wait relay (leader);
+// warp 7 P forwarder (both).  The softmax warps announce P on a local mbarrier (cheap);
+// the forwarder of each CTA waits on it and does the one cluster-scope release add per
+// tile on a counter in the leader's shared memory, which the MMA thread polls -- a
+// cluster-scope release costs ~450 cycles, too much to pay on the softmax warps' path.
+//
+// The last, partial key tile of a range is read as the window [k_end - 128, k_end):
+// every row copied is a valid key (or a zero-filled row at a negative coordinate), and
+// the columns that belong to earlier tiles or ranges are masked by selection, so key
+// padding is never read.
+
+struct PairCfg {
+    static constexpr int D = 256;
+    static constexpr int ROWS = 128;                 // query rows per CTA (TMEM lanes)
+    static constexpr int NBLK = D / 64;              // 64-column (128-byte) blocks per row
+    static constexpr int Q_BYTES = ROWS * D * 2;     // 64 KB
+    static constexpr int KH = BN / 2;                // keys of a K tile held by one CTA
+    static constexpr int KBLK_BYTES = KH * 128;      // one 64-column block of them: 8 KB
+    static constexpr int VBLK_BYTES = BN * 128;      // one 64-column block of V: 16 KB
+    static constexpr int SLOT = 32768;               // one CTA's half of a K or V tile
+    static constexpr int CTRL = 1024;
+    static constexpr int NSLOTS = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
+    static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
+    static constexpr int THREADS = 256;
+    static_assert(NSLOTS >= 4 && NSLOTS <= 8, "pair ring depth");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "pair shared memory budget");
+    static_assert(NBLK * KBLK_BYTES == SLOT && (NBLK / 2) * VBLK_BYTES == SLOT, "half tiles fill a slot");
+};
+
+enum : int {
+    PB_Q = 0,
+    PB_FULL = 1,     // [8] slot filled by both CTAs' copies (leader)
+    PB_EMPTY = 9,    // [8] slot consumed (multicast commit, both CTAs)
+    PB_S = 17,       // [2] S_j ready (multicast commit, both CTAs)
+    PB_O = 19,       // PV of the last two tiles complete (multicast commit, both CTAs)
+    PB_DRAIN = 20,   // leader only
+    PB_PL = 21,      // [2] P_j stored by this CTA's softmax warps (4 warp arrivals)
+    PB_NUM = 23
+};
+
+template <bool SPLIT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    using C = PairCfg;
+    constexpr int D = C::D;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // Swizzled tiles need 1024-byte alignment; both CTAs see the same layout, so both
+    // return here together (no cluster barrier has been reached yet).
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(&g_attn_status, STATUS_LAYOUT);
+        return;
+    }
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + C::Q_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::NSLOTS * C::SLOT);
+    uint32_t* words = reinterpret_cast<uint32_t*>(bars + PB_NUM);   // tmem, abort, relay seq, P count
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
+    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t sQ_addr = smem_u32(sQ);
+    const uint32_t sKV_addr = smem_u32(sKV);
+    const uint32_t seq_addr = smem_u32(words + 2);
+    const uint32_t pcnt_addr = smem_u32(words + 3);
+#define PBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    // ---- work unit of the pair: 256-row query tile fastest, then split chunk, then (b, h)
+    int unit = static_cast<int>(blockIdx.x >> 1);
+    const int ptile = unit % p.n_qtiles;
+    unit /= p.n_qtiles;
+    const int split = SPLIT ? unit % p.num_splits : 0;
+    const int bh = SPLIT ? unit / p.num_splits : unit;
+    const int b = bh / p.H;
+    const int q0 = ptile * (2 * C::ROWS) + static_cast<int>(rank) * C::ROWS;
+
+    int kv = __ldg(p.kv_len + b);
+    if (kv < 0 || kv > p.Tk) {
+        if (tid == 0 && leader) atomicOr(&g_attn_status, STATUS_KVLEN);
+        kv = kv < 0 ? 0 : p.Tk;
+    }
+    const int k_begin = SPLIT ? split * p.chunk_len : 0;
+    const int k_end = SPLIT ? min(kv, k_begin + p.chunk_len) : kv;
+    const int n_tiles = (k_end > k_begin) ? (k_end - k_begin + BN - 1) / BN : 0;
+    // leading columns of the last tile that belong to earlier tiles (0 when it is full)
+    const int last_lo = n_tiles > 0 ? n_tiles * BN - (k_end - k_begin) : 0;
+    auto tile_key0 = [&](int j) { return (j == n_tiles - 1 && last_lo > 0) ? k_end - BN : k_begin + j * BN; };
+
+    if (tid == 0) {
+        mbar_init(PBAR(PB_Q), 1);
+        for (int s = 0; s < C::NSLOTS; ++s) {
+            mbar_init(PBAR(PB_FULL + s), 1);
+            mbar_init(PBAR(PB_EMPTY + s), 1);
+        }
+        mbar_init(PBAR(PB_S + 0), 1);
+        mbar_init(PBAR(PB_S + 1), 1);
+        mbar_init(PBAR(PB_O), 1);
+        mbar_init(PBAR(PB_DRAIN), 1);
+        mbar_init(PBAR(PB_PL + 0), 4);
+        mbar_init(PBAR(PB_PL + 1), 4);
+        words[1] = 0u;
+        words[2] = 0u;
+        words[3] = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc_pair(smem_u32(words), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = words[0];
+    const unsigned long long wlim = p.wait_ns;
+
+    if (warp == 4) {
+        // ================================================================ producer (both CTAs)
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_map(&tm_q);
+            tma_prefetch_map(&tm_k);
+            tma_prefetch_map(&tm_v);
+            if (leader) mbar_arrive_expect_tx(PBAR(PB_Q), 2 * C::Q_BYTES);
+            const uint32_t lq = mapa_shared(PBAR(PB_Q), 0);
+#pragma unroll
+            for (int blk = 0; blk < C::NBLK; ++blk)
+                tma_load_3d_pair(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, bh, lq);
+            int slot = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            auto item = [&](bool is_k, int j) {
+                if (!ok) return;
+                ok = wait_bar_cl(PBAR(PB_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
+                if (!ok) return;
+                if (leader) mbar_arrive_expect_tx(PBAR(PB_FULL + slot), 2 * C::SLOT);
+                const uint32_t lfull = mapa_shared(PBAR(PB_FULL + slot), 0);
+                const uint32_t dst = sKV_addr + slot * C::SLOT;
+                const int key0 = tile_key0(j);
+                if (is_k) {
+                    const bool drop = (p.debug & ATTN_DEBUG_DROP_COPY) && leader && j == 0;
+#pragma unroll
+                    for (int c = 0; c < C::NBLK; ++c)
+                        if (!(drop && c == 0))
+                            tma_load_3d_pair(dst + c * C::KBLK_BYTES, &tm_k, c * 64, key0 + static_cast<int>(rank) * C::KH,
+                                             bh, lfull);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < C::NBLK / 2; ++c)
+                        tma_load_3d_pair(dst + c * C::VBLK_BYTES, &tm_v, static_cast<int>(rank) * (D / 2) + c * 64,
+                                         key0, bh, lfull);
+                }
+                if (++slot == C::NSLOTS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            };
+            item(true, 0);
+            if (n_tiles > 1) item(true, 1);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                item(false, j);
+                if (j + 2 < n_tiles) item(true, j + 2);
+            }
+            if (!ok) {
+                // Copies already issued complete on the leader's barriers; give them time to
+                // land before this CTA's memory can be reused.
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 2000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // ================================================================ wait relay (leader)
+        // Waits on Q and on every slot in consumption order (K_0, K_1, then V_j, K_{j+2})
+        // and publishes the count of completed events with a release store.
+        if (leader && lane == 0 && n_tiles > 0) {
+            uint32_t seq = 0;
+            bool ok = wait_bar_cl(PBAR(PB_Q), 0, abort_flag, wlim);
+            if (ok) st_release_smem(seq_addr, ++seq);
+            int slot = 0;
+            uint32_t phase = 0;
+            const int items = 2 * n_tiles;
+#pragma unroll 1
+            for (int i = 0; i < items && ok; ++i) {
+                ok = wait_bar_cl(PBAR(PB_FULL + slot), phase, abort_flag, wlim);
+                if (!ok) break;
+                st_release_smem(seq_addr, ++seq);
+                if (++slot == C::NSLOTS) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ================================================================ MMA issuer (leader)
+        if (leader && lane == 0 && n_tiles > 0) {
+            constexpr uint32_t IDESC_S = make_idesc_bf16(2 * C::ROWS, BN, false);
+            constexpr uint32_t IDESC_PV = make_idesc_bf16(2 * C::ROWS, D, true);
+            const uint64_t q_desc0 = make_smem_desc(sQ_addr, 16, 1024, 2);
+            const uint64_t k_desc0 = make_smem_desc(sKV_addr, 16, 1024, 2);
+            const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::VBLK_BYTES, 1024, 2);
+            int slot = 0;
+            uint32_t consumed = 0;
+            auto poll_ge = [&](uint32_t addr, uint32_t need) -> bool {
+                if (ld_acquire_cluster_smem(addr) >= need) return true;
+                const uint64_t t0 = global_timer_ns();
+                while (true) {
+                    if (ld_acquire_cluster_smem(addr) >= need) return true;
+                    if (*abort_flag) return false;
+                    if (global_timer_ns() - t0 > wlim) {
+                        *abort_flag = 1;
+                        atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                        return false;
+                    }
+                }
+            };
+            auto slot_desc = [&](uint64_t d0) { return d0 + static_cast<uint64_t>(slot) * (C::SLOT >> 4); };
+            auto next_slot = [&]() { slot = (slot + 1 == C::NSLOTS) ? 0 : slot + 1; };
+            bool ok = poll_ge(seq_addr, ++consumed);   // both Q tiles landed
+            auto issue_s = [&](int j) {
+                ok = poll_ge(seq_addr, ++consumed);     // K_j halves landed in both CTAs
+                if (!ok) return;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+                const uint64_t kd = slot_desc(k_desc0);
+#pragma unroll
+                for (int t = 0; t < D / 16; ++t) {
+                    const int c = t >> 2, kk = t & 3;
+                    mma_ss_pair(d_tmem, q_desc0 + static_cast<uint64_t>(((c * C::ROWS * 128) >> 4) + kk * 2),
+                                kd + static_cast<uint64_t>(((c * C::KBLK_BYTES) >> 4) + kk * 2), IDESC_S, t != 0);
+                }
+                tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
+                tc_commit_pair(PBAR(PB_S + (j & 1)), 0x3);
+                next_slot();
+            };
+            auto issue_pv = [&](int j) {
+                ok = poll_ge(pcnt_addr, 2u * static_cast<uint32_t>(j + 1));   // P_j stored in both CTAs
+                if (!ok) return;
+                ok = poll_ge(seq_addr, ++consumed);                        // V_j halves landed
+                if (!ok) return;
+                tc_fence_after();
+                const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+                const uint64_t vd = slot_desc(v_desc0);
+#pragma unroll
+                for (int kb = 0; kb < BN / 16; ++kb)
+                    mma_ts_pair(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV,
+                                (j == 0 && kb == 0) ? 0u : 1u);
+                tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
+                if (j >= n_tiles - 2) tc_commit_pair(PBAR(PB_O), 0x3);
+                next_slot();
+            };
+            if (ok) issue_s(0);
+            if (ok && n_tiles > 1) issue_s(1);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                issue_pv(j);
+                if (ok && j + 2 < n_tiles) issue_s(j + 2);
+            }
+            tc_commit_pair(PBAR(PB_DRAIN), 0x1);
+            wait_bar_drain_cl(PBAR(PB_DRAIN), 0, wlim);
+        }
+        __syncwarp();
+    } else if (warp == 7) {
+        // ================================================================ P forwarder (both CTAs)
+        if (lane == 0 && n_tiles > 0) {
+            const uint32_t lead_pcnt = mapa_shared(pcnt_addr, 0);
+#pragma unroll 1
+            for (int j = 0; j < n_tiles; ++j) {
+                if (!wait_bar_cl(PBAR(PB_PL + (j & 1)), (j >> 1) & 1, abort_flag, wlim)) break;
+                red_add_release_cluster(lead_pcnt, 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ================================================================ softmax (both CTAs)
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        const bool pos_scale = sl2 > 0.0f;
+        float m_ref = -INFINITY;
+        float l_sum = 0.0f;
+        bool ok = true;
+#pragma unroll 1
+        for (int j = 0; j < n_tiles; ++j) {
+            ok = __all_sync(0xffffffffu, wait_bar_cl(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
+            uint32_t raw[BN];
+            tmem_ld128_wait(s_addr, raw);
+            float x[BN];
+            const int lo = (j == n_tiles - 1) ? last_lo : 0;   // columns [0, lo) are not this tile's keys
+            if (lo > 0) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(raw[c]);
+            }
+            if (!pos_scale) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
+            }
+            float mxp[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) mxp[t] = x[t];
+#pragma unroll
+            for (int c = 8; c < BN; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) *
+                             (pos_scale ? sl2 : 1.0f);
+            float factor = 1.0f;
+            bool rescale = false;
+            if (j == 0) {
+                m_ref = mx;
+            } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
+                const float m_new = fmaxf(m_ref, mx);
+                factor = fast_exp2(m_ref - m_new);
+                m_ref = m_new;
+                rescale = true;
+            }
+            const float mul = pos_scale ? sl2 : 1.0f;
+            const float neg_m = -m_ref;
+            float sp[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
+                    const float p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
+                    sp[e & 7] += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(s_addr + cc * 16, pk);
+            }
+            const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            l_sum = l_sum * factor + tile_sum;
+            if (rescale) {
+                // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last tile
+                // the leader announces PV_{n-2} on the O barrier.
+                const bool w = (j + 1 < n_tiles)
+                                   ? wait_bar_cl(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
+                                   : wait_bar_cl(PBAR(PB_O), 0, abort_flag, wlim);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int oc = 0; oc < D / 32; ++oc) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                    tmem_st32(tmem + lane_base + O_COL + oc * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(PBAR(PB_PL + (j & 1)));
+        }
+        // ---- epilogue
+        if (ok && n_tiles > 0) {
+            bool w = wait_bar_cl(PBAR(PB_O), 0, abort_flag, wlim);
+            if (n_tiles > 1) w = w && wait_bar_cl(PBAR(PB_O), 1, abort_flag, wlim);
+            ok = __all_sync(0xffffffffu, w);
+            tc_fence_after();
+        }
+        const int row = q0 + tid;
+        const bool in_range = row < p.Tq;
+        const bool have = n_tiles > 0;
+        const float inv_l = have ? 1.0f / l_sum : 0.0f;
+        const float lse_val = have ? (m_ref + log2f(l_sum)) * LN2 : -INFINITY;
+        const long long BH = static_cast<long long>(p.B) * p.H;
+#pragma unroll 1
+        for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t o[32];
+            if (have) {
+                tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            if (!in_range) continue;
+            if constexpr (SPLIT) {
+                float* dst = p.part_out + ((static_cast<long long>(split) * BH + bh) * p.Tq + row) * D + oc * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    float4 v4 = make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                                            __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+                    *reinterpret_cast<float4*>(dst + e) = v4;
+                }
+            } else {
+                __nv_bfloat16* dst = p.out + (static_cast<long long>(bh) * p.Tq + row) * D + oc * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 v4;
+                    v4.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+                    v4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+                    v4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+                    v4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+                    *reinterpret_cast<uint4*>(dst + e) = v4;
+                }
+            }
+        }
+        if (in_range) {
+            if constexpr (SPLIT) {
+                p.part_lse[(static_cast<long long>(split) * BH + bh) * p.Tq + row] = lse_val;
+            } else if (p.lse != nullptr) {
+                p.lse[static_cast<long long>(bh) * p.Tq + row] = lse_val;
+            }
+        }
+    }
+
+    // Neither CTA may release its TMEM or leave while the pair's MMAs, commits or copies
+    // may still touch the other one.
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+#undef PBAR
+}
