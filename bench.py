@@ -245,6 +245,10 @@ def run_ours(args, rank, world):
     peaks, peaks_src = load_peaks()
     kern_avg_ms = statistics.mean(kern_ms)
     achieved = flops / (kern_avg_ms * 1e-3) / 1e12
+    # the dominant kernel: head dim 256 runs on CTA pairs, others on single CTAs
+    kernel_tag = "attn_fwd_pair" if w.D == 256 else f"attn_fwd_d{w.D}"
+    kernel_name = (f"attn_fwd_pair_kernel<{int(bool(splits))}>" if w.D == 256
+                   else f"attn_fwd_kernel<{w.D},{int(bool(splits))}>")
     peak_key = "bf16_tflops_sustained"
     peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
     roofline = {
@@ -252,8 +256,8 @@ def run_ours(args, rank, world):
         "frac": round(achieved / peak, 4),
         "peak_source": f"{peaks_src} {peak_key} (kernel timed inside a seconds-long back-to-back loop)",
         "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
-        "traffic": traffic_from_profile(args.workload),
-        "kernel": "attn_fwd_kernel<256,split>" if splits else f"attn_fwd_kernel<{w.D},single>",
+        "traffic": traffic_from_profile(args.workload, kernel_tag),
+        "kernel": kernel_name,
     }
     rec = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -346,9 +350,9 @@ def verify_rows(case, out, lse, w):
             "max_abs_err_out": float(np.abs(go - ro).max())}
 
 
-def traffic_from_profile(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this kernel, if any."""
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+def traffic_from_profile(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and workload."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.json")
     try:
         with open(path) as f:
             return json.load(f).get("dram_bytes_per_launch")
