@@ -9,13 +9,14 @@
 // tile instead of 128 KB: the five 32 KB ring slots hold 2.5 tiles of look-ahead, which
 // takes the copy latency off the critical path.
 //
-// Roles (256 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
+// Roles (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
 // producer (both CTAs, into their own memory, completing on the leader's barriers);
-// warp 5 TMEM allocation (both) and MMA issue (leader); warp 6 wait relay (leader);
-// warp 7 P forwarder (both).  The softmax warps announce P on a local mbarrier (cheap);
-// the forwarder of each CTA waits on it and does the one cluster-scope release add per
-// tile on a counter in the leader's shared memory, which the MMA thread polls -- a
-// cluster-scope release costs ~450 cycles, too much to pay on the softmax warps' path.
+// warp 5 TMEM allocation (both) and MMA issue (leader); warp 6 wait relay (leader).
+// Each softmax warp of either CTA announces P with one arrival on the leader's P
+// barrier (the remote mbarrier arrive with default semantics -- release at CTA scope --
+// which is the cross-CTA handshake the pair pipelines are built on; a cluster-scope
+// release costs ~450-1100 cycles and made this handshake the critical path).  The relay
+// folds "P_j stored in both CTAs" and "V_j landed" into one event for the MMA thread.
 //
 // The last, partial key tile of a range is read as the window [k_end - 128, k_end):
 // every row copied is a valid key (or a zero-filled row at a negative coordinate), and
@@ -34,7 +35,7 @@ struct PairCfg {
     static constexpr int CTRL = 1024;
     static constexpr int NSLOTS = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
     static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
-    static constexpr int THREADS = 256;
+    static constexpr int THREADS = 224;
     static_assert(NSLOTS >= 4 && NSLOTS <= 8, "pair ring depth");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "pair shared memory budget");
     static_assert(NBLK * KBLK_BYTES == SLOT && (NBLK / 2) * VBLK_BYTES == SLOT, "half tiles fill a slot");
@@ -47,7 +48,7 @@ enum : int {
     PB_S = 17,       // [2] S_j ready (multicast commit, both CTAs)
     PB_O = 19,       // PV of the last two tiles complete (multicast commit, both CTAs)
     PB_DRAIN = 20,   // leader only
-    PB_PL = 21,      // [2] P_j stored by this CTA's softmax warps (4 warp arrivals)
+    PB_P = 21,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
     PB_NUM = 23
 };
 
@@ -67,13 +68,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::Q_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::NSLOTS * C::SLOT);
-    uint32_t* words = reinterpret_cast<uint32_t*>(bars + PB_NUM);   // tmem, abort, relay seq, P count
+    uint32_t* words = reinterpret_cast<uint32_t*>(bars + PB_NUM);   // tmem, abort, relay seq
     volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
     const uint32_t bar0 = smem_u32(bars);
     const uint32_t sQ_addr = smem_u32(sQ);
     const uint32_t sKV_addr = smem_u32(sKV);
     const uint32_t seq_addr = smem_u32(words + 2);
-    const uint32_t pcnt_addr = smem_u32(words + 3);
 #define PBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
     const int tid = threadIdx.x;
@@ -113,11 +113,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         mbar_init(PBAR(PB_S + 1), 1);
         mbar_init(PBAR(PB_O), 1);
         mbar_init(PBAR(PB_DRAIN), 1);
-        mbar_init(PBAR(PB_PL + 0), 4);
-        mbar_init(PBAR(PB_PL + 1), 4);
+        mbar_init(PBAR(PB_P + 0), 8);
+        mbar_init(PBAR(PB_P + 1), 8);
         words[1] = 0u;
         words[2] = 0u;
-        words[3] = 0u;
         fence_mbar_init();
     }
     if (warp == 5) {
@@ -146,7 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             bool ok = true;
             auto item = [&](bool is_k, int j) {
                 if (!ok) return;
-                ok = wait_bar_cl(PBAR(PB_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
+                ok = wait_bar(PBAR(PB_EMPTY + slot), phase ^ 1u, abort_flag, wlim);
                 if (!ok) return;
                 if (leader) mbar_arrive_expect_tx(PBAR(PB_FULL + slot), 2 * C::SLOT);
                 const uint32_t lfull = mapa_shared(PBAR(PB_FULL + slot), 0);
@@ -188,23 +187,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         __syncwarp();
     } else if (warp == 6) {
         // ================================================================ wait relay (leader)
-        // Waits on Q and on every slot in consumption order (K_0, K_1, then V_j, K_{j+2})
-        // and publishes the count of completed events with a release store.
+        // Waits on Q and, in the MMA thread's consumption order, on K_0, K_1, then per tile
+        // "P_j stored in both CTAs and V_j landed" and K_{j+2}; publishes the count of
+        // completed events with a release store.
         if (leader && lane == 0 && n_tiles > 0) {
             uint32_t seq = 0;
-            bool ok = wait_bar_cl(PBAR(PB_Q), 0, abort_flag, wlim);
+            bool ok = wait_bar(PBAR(PB_Q), 0, abort_flag, wlim);
             if (ok) st_release_smem(seq_addr, ++seq);
             int slot = 0;
             uint32_t phase = 0;
-            const int items = 2 * n_tiles;
-#pragma unroll 1
-            for (int i = 0; i < items && ok; ++i) {
-                ok = wait_bar_cl(PBAR(PB_FULL + slot), phase, abort_flag, wlim);
-                if (!ok) break;
-                st_release_smem(seq_addr, ++seq);
+            auto item = [&]() {
+                ok = ok && wait_bar(PBAR(PB_FULL + slot), phase, abort_flag, wlim);
                 if (++slot == C::NSLOTS) {
                     slot = 0;
                     phase ^= 1u;
+                }
+            };
+            auto publish = [&]() {
+                if (ok) st_release_smem(seq_addr, ++seq);
+            };
+            item();  // K_0
+            publish();
+            if (n_tiles > 1) {
+                item();  // K_1
+                publish();
+            }
+#pragma unroll 1
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                ok = wait_bar(PBAR(PB_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                item();  // V_j
+                publish();
+                if (j + 2 < n_tiles) {
+                    item();  // K_{j+2}
+                    publish();
                 }
             }
         }
@@ -252,9 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 next_slot();
             };
             auto issue_pv = [&](int j) {
-                ok = poll_ge(pcnt_addr, 2u * static_cast<uint32_t>(j + 1));   // P_j stored in both CTAs
-                if (!ok) return;
-                ok = poll_ge(seq_addr, ++consumed);                        // V_j halves landed
+                ok = poll_ge(seq_addr, ++consumed);   // P_j stored in both CTAs and V_j halves landed
                 if (!ok) return;
                 tc_fence_after();
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
@@ -276,18 +289,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 if (ok && j + 2 < n_tiles) issue_s(j + 2);
             }
             tc_commit_pair(PBAR(PB_DRAIN), 0x1);
-            wait_bar_drain_cl(PBAR(PB_DRAIN), 0, wlim);
-        }
-        __syncwarp();
-    } else if (warp == 7) {
-        // ================================================================ P forwarder (both CTAs)
-        if (lane == 0 && n_tiles > 0) {
-            const uint32_t lead_pcnt = mapa_shared(pcnt_addr, 0);
-#pragma unroll 1
-            for (int j = 0; j < n_tiles; ++j) {
-                if (!wait_bar_cl(PBAR(PB_PL + (j & 1)), (j >> 1) & 1, abort_flag, wlim)) break;
-                red_add_release_cluster(lead_pcnt, 1u);
-            }
+            wait_bar_drain(PBAR(PB_DRAIN), 0, wlim);
         }
         __syncwarp();
     } else if (warp < 4) {
@@ -300,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         bool ok = true;
 #pragma unroll 1
         for (int j = 0; j < n_tiles; ++j) {
-            ok = __all_sync(0xffffffffu, wait_bar_cl(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+            ok = __all_sync(0xffffffffu, wait_bar(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
@@ -360,8 +362,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last tile
                 // the leader announces PV_{n-2} on the O barrier.
                 const bool w = (j + 1 < n_tiles)
-                                   ? wait_bar_cl(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
-                                   : wait_bar_cl(PBAR(PB_O), 0, abort_flag, wlim);
+                                   ? wait_bar(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
+                                   : wait_bar(PBAR(PB_O), 0, abort_flag, wlim);
                 ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
                 tc_fence_after();
@@ -377,12 +379,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(PBAR(PB_PL + (j & 1)));
+            if (lane == 0) mbar_arrive_remote(mapa_shared(PBAR(PB_P + (j & 1)), 0));
         }
         // ---- epilogue
         if (ok && n_tiles > 0) {
-            bool w = wait_bar_cl(PBAR(PB_O), 0, abort_flag, wlim);
-            if (n_tiles > 1) w = w && wait_bar_cl(PBAR(PB_O), 1, abort_flag, wlim);
+            bool w = wait_bar(PBAR(PB_O), 0, abort_flag, wlim);
+            if (n_tiles > 1) w = w && wait_bar(PBAR(PB_O), 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }

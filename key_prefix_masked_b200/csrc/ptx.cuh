@@ -186,6 +186,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
         : "memory");
     return ok != 0;
 }
+// Arrival on an mbarrier in another CTA of the cluster (default semantics: release at
+// CTA scope, the form the CUDA pair pipelines use for cross-CTA handshakes).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
 // Atomic add with cluster-scope release on a word in (possibly another CTA's) shared memory.
 __device__ __forceinline__ void red_add_release_cluster(uint32_t cluster_addr, uint32_t v) {
     asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;\n" ::"r"(cluster_addr), "r"(v) : "memory");
