@@ -57,6 +57,11 @@ def workload_flops(w: synth.Workload, kv_list) -> float:
     return float(sum(4.0 * w.H * w.Tq * n * w.D for n in kv_list))
 
 
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Throughput of the whole job: every rank's work over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ distributed plumbing
 def dist_setup(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -232,7 +237,7 @@ def run_ours(args, rank, world):
     kern_ms = ([a.elapsed_time(b_) for a, b_ in k_ev] if k_ev else step_ms)
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms_per_step)
 
     # ---- end-to-end: pinned host buffers, copies inside the timed region
     e2e = run_e2e(kp, w, case, scale, splits, args, world)

@@ -26,9 +26,10 @@
 //               by more than 2^8 (exact either way: O and the row sum always share one
 //               reference max).  At the end O is divided by the row sum and written as
 //               bf16 (fp32 for split partials) with lse = ln(sum) + max.
-// In the last, partial key tile the value rows between kv_len and the next multiple of
-// 16 are zeroed in shared memory before the PV MMA, and MMA steps lying wholly past
-// kv_len are skipped, so padding content (NaN included) never reaches an accumulator.
+// The last, partial key tile of a range is read as the window [k_end - 128, k_end): every
+// row copied is a valid key (or a zero-filled row at a negative coordinate) and the
+// columns that belong to earlier tiles are masked by selection, so key padding (NaN
+// included) is never even read.
 //
 // Every mbarrier wait is bounded (%globaltimer); on expiry the CTA raises a sticky
 // device flag, drains its copies and MMAs in flight, frees its TMEM and exits.
@@ -223,6 +224,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int k_begin = SPLIT ? split * p.chunk_len : 0;
     const int k_end = SPLIT ? min(kv, k_begin + p.chunk_len) : kv;
     const int n_tiles = (k_end > k_begin) ? (k_end - k_begin + BN - 1) / BN : 0;
+    // The last, partial tile is read as the window [k_end - BN, k_end); its leading
+    // last_lo columns belong to earlier tiles (or precede the range) and are masked.
+    const int last_lo = n_tiles > 0 ? n_tiles * BN - (k_end - k_begin) : 0;
+    auto tile_key0 = [&](int j) { return (j == n_tiles - 1 && last_lo > 0) ? k_end - BN : k_begin + j * BN; };
 
     if (tid == 0) {
         mbar_init(BAR(BAR_Q), 1);
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             };
             auto load_k = [&](int j) {
-                const int key0 = k_begin + j * BN;
+                const int key0 = tile_key0(j);
 #pragma unroll 1
                 for (int g = 0; g < C::KCH / C::GRP && ok; ++g) {
                     if (!acquire()) break;
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             };
             auto load_v = [&](int j) {
-                const int key0 = k_begin + j * BN;
+                const int key0 = tile_key0(j);
 #pragma unroll 1
                 for (int g = 0; g < C::VCH / C::GRP && ok; ++g) {
                     if (!acquire()) break;
@@ -392,56 +397,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 advance(KG);
             };
             auto issue_pv = [&](int j) {
-                const int valid = min(BN, k_end - (k_begin + j * BN));
+                // Every 16-key step is issued, partial last tile included: its masked
+                // columns hold P = 0 against value rows that are valid keys of earlier
+                // tiles (or zero fill), never padding.
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
-                if (valid == BN) {
-                    const uint32_t acc0 = (j == 0) ? 0u : 1u;
+                const uint32_t acc0 = (j == 0) ? 0u : 1u;
 #pragma unroll
-                    for (int g = 0; g < VG; ++g) {
-                        const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
+                for (int g = 0; g < VG; ++g) {
+                    const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
 #pragma unroll
-                        for (int cc = 0; cc < C::GRP; ++cc) {
+                    for (int cc = 0; cc < C::GRP; ++cc) {
 #pragma unroll
-                            for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
-                                const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
-                                mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                       vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
-                                       IDESC_PV, kb == 0 ? acc0 : 1u);
-                            }
-                        }
-                    }
-                } else {
-                    // Partial tile: zero the value rows in [valid, 16*kblocks) and skip the
-                    // 16-key steps that hold no valid key.
-                    const int kblocks = (valid + 15) >> 4;
-                    bool wrote = false;
-                    for (int g = 0; g < VG; ++g) {
-                        for (int cc = 0; cc < C::GRP; ++cc) {
-                            const int c = g * C::GRP + cc;
-                            const int r0 = max(valid, c * C::V_ROWS);
-                            const int r1 = min(kblocks * 16, (c + 1) * C::V_ROWS);
-                            uint8_t* vs = sKV + (ring(g) * C::GRP + cc) * C::SLOT;
-                            for (int r = r0; r < r1; ++r)
-                                for (int blk = 0; blk < C::NBLK; ++blk)
-                                    for (int piece = 0; piece < C::SW / 16; ++piece) {
-                                        *reinterpret_cast<uint4*>(vs + blk * C::V_ROWS * C::SW +
-                                                                  (r - c * C::V_ROWS) * C::SW + piece * 16) =
-                                            make_uint4(0u, 0u, 0u, 0u);
-                                        wrote = true;
-                                    }
-                        }
-                    }
-                    if (wrote) fence_proxy_async_smem();
-                    for (int g = 0; g < VG; ++g) {
-                        const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
-                        for (int cc = 0; cc < C::GRP; ++cc) {
-                            for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
-                                const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
-                                if (kb < kblocks)
-                                    mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                           vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
-                                           IDESC_PV, (j == 0 && kb == 0) ? 0u : 1u);
-                            }
+                        for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
+                            const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
+                            mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                   vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
+                                   IDESC_PV, kb == 0 ? acc0 : 1u);
                         }
                     }
                 }
@@ -534,18 +505,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t raw[BN];
             tmem_ld128_wait(s_addr, raw);
             float x[BN];
-            const int valid = min(BN, k_end - (k_begin + j * BN));
-            if (valid < BN) {
+            const int lo = (j == n_tiles - 1) ? last_lo : 0;   // columns [0, lo) are not this tile's keys
+            if (lo > 0) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) x[c] = (c < valid) ? __uint_as_float(raw[c]) : -INFINITY;
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
             } else {
 #pragma unroll
                 for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(raw[c]);
             }
             if (!pos_scale) {
-                // zero or negative scale: scale every finite score first (the max flips)
+                // zero or negative scale: scale every valid score first (the max flips)
 #pragma unroll
-                for (int c = 0; c < BN; ++c) x[c] = (c < valid) ? x[c] * sl2 : -INFINITY;
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
             }
             // tree max over the row
             float mxp[8];
