@@ -51,7 +51,6 @@ namespace attn {
 
 constexpr int BM = 128;               // query rows per CTA (one TMEM lane each)
 constexpr int BN = 128;               // keys per tile
-constexpr int NUM_THREADS = 224;      // 4 softmax warps + producer + MMA issuer + wait relay
 constexpr int SMEM_LIMIT = 232448;    // 227 KB opt-in dynamic shared memory per block
 constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128) S1 [128,256) O [256, 256+D)
 constexpr uint32_t O_COL = 256;
@@ -73,12 +72,21 @@ struct Cfg {
     static constexpr int KCH = NBLK;                  // K tile: one chunk per column block
     static constexpr int VCH = NBLK;                  // V tile: chunks of V_ROWS key rows
     static constexpr int V_ROWS = BN / VCH;
-    static constexpr int NSLOTS_RAW = (SMEM_LIMIT - Q_BYTES - 2048) / SLOT;
+    // Head dims whose two O accumulators fit in TMEM beside the two S buffers run two
+    // softmax warpgroups (even and odd key tiles); larger ones run one.
+    static constexpr bool DUAL = O_COL + 2 * D <= TMEM_COLS;
+    static constexpr int SM_WARPS = DUAL ? 8 : 4;
+    static constexpr int WARP_PROD = SM_WARPS;          // TMA producer
+    static constexpr int WARP_MMA = SM_WARPS + 1;       // MMA issuer, TMEM owner
+    static constexpr int WARP_RELAY = SM_WARPS + 2;     // wait relay
+    static constexpr int THREADS = 32 * (SM_WARPS + 3);
+    static constexpr int XCH_BYTES = DUAL ? 2 * 2 * BM * 4 : 0;   // per-group (max, sum) exchange
+    static constexpr int NSLOTS_RAW = (SMEM_LIMIT - Q_BYTES - 2048 - XCH_BYTES) / SLOT;
     static constexpr int GRP = (KCH >= 2) ? 2 : 1;      // chunks per ring group (one barrier pair)
     static constexpr int NSLOTS_CAP = NSLOTS_RAW > 16 ? 16 : NSLOTS_RAW;
     static constexpr int NSLOTS = NSLOTS_CAP / GRP * GRP;
     static constexpr int NG = NSLOTS / GRP;             // ring groups
-    static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOTS * SLOT + 1024;
+    static constexpr int SMEM_BYTES = 1024 + Q_BYTES + NSLOTS * SLOT + 1024 + XCH_BYTES;
     static constexpr uint32_t LAYOUT = (SW == 128) ? 2u : 4u;
     static_assert(D % BLK == 0, "head dim must be a multiple of the swizzle block");
     static_assert(V_ROWS % 16 == 0, "value chunks must hold whole 16-key MMA steps");
@@ -93,7 +101,7 @@ enum : int {
     BAR_FULL = 1,       // [16] ring group filled (TMA tx)
     BAR_EMPTY = 17,     // [16] ring group consumed (tcgen05.commit)
     BAR_S = 33,         // [2] S_j ready in TMEM buffer j&1
-    BAR_P = 35,         // [2] P_j stored over S_j (128 softmax arrivals)
+    BAR_P = 35,         // [2] P_j stored over S_j (one arrival per softmax warp of its group)
     BAR_O = 37,         // PV complete, announced for the last two tiles only
     BAR_DRAIN = 39,
     NUM_BARS = 40
@@ -184,7 +192,7 @@ __device__ __noinline__ bool wait_bar_drain_cl(uint32_t bar, uint32_t parity, un
 }
 
 template <int D, bool SPLIT>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
     using C = Cfg<D>;
@@ -237,7 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(BAR_S + i), 1);
-            mbar_init(BAR(BAR_P + i), 128);
+            mbar_init(BAR(BAR_P + i), 4);
         }
         mbar_init(BAR(BAR_O), 1);
         mbar_init(BAR(BAR_DRAIN), 1);
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *ready_seq = 0u;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
         tmem_relinquish();
     }
@@ -255,7 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem = *tmem_holder;
     const unsigned long long wlim = p.wait_ns;
 
-    if (warp == 4) {
+    if (warp == C::WARP_PROD) {
         // ================================================================ producer
         // Loads go out in the order the MMA thread consumes them: K_0, K_1, then
         // V_j, K_{j+2} for every tile j.  Each tile half is GRP-chunk groups; one ring
@@ -337,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == C::WARP_MMA) {
         // ================================================================ MMA issuer (one thread)
         // Two readiness events per tile, published by the relay warp: "P_j stored and
         // V_j landed" and "K_{j+2} landed".  Between them the 8 PV and 16 S MMAs of a
@@ -400,8 +408,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // Every 16-key step is issued, partial last tile included: its masked
                 // columns hold P = 0 against value rows that are valid keys of earlier
                 // tiles (or zero fill), never padding.
+                // Two accumulators (DUAL): PV_j adds into O_{j&1}; each starts fresh.
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
-                const uint32_t acc0 = (j == 0) ? 0u : 1u;
+                const uint32_t o_tmem = tmem + O_COL + (C::DUAL ? static_cast<uint32_t>((j & 1) * D) : 0u);
+                const uint32_t acc0 = (j < (C::DUAL ? 2 : 1)) ? 0u : 1u;
 #pragma unroll
                 for (int g = 0; g < VG; ++g) {
                     const uint64_t vd = v_desc0 + static_cast<uint64_t>(ring(g)) * GSTEP;
@@ -410,7 +420,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                         for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
                             const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
-                            mma_ts(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                            mma_ts(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
                                    vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
                                    IDESC_PV, kb == 0 ? acc0 : 1u);
                         }
@@ -454,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             wait_bar_drain(BAR(BAR_DRAIN), 0, wlim);
         }
         __syncwarp();
-    } else if (warp == 6) {
+    } else if (warp == C::WARP_RELAY) {
         // ================================================================ wait relay
         // Waits on the ring groups and P barriers in the MMA thread's consumption order
         // and publishes one completed event per MMA batch with a release store: K_0,
@@ -490,14 +500,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else {
         // ================================================================ softmax
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // Thread t of warpgroup w (warps 4w .. 4w+3) owns query row r = t % 128 (TMEM lane r).
+        // Head dims up to 64 (DUAL): warpgroup w takes the key tiles j = w (mod 2) with its
+        // own running max, row sum and O accumulator (TMEM columns O_COL + w*D), so one
+        // group's max phase overlaps the other's exponentials; the two partial results are
+        // combined exactly at the end (the log-sum-exp rule of split-KV).  Head dim 256
+        // (test hook only) keeps one accumulator and warpgroup 0 takes every tile.
+        constexpr bool DUAL = C::DUAL;
+        const int wg = warp >> 2;
+        const int r = tid & 127;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t o_col = O_COL + (DUAL ? static_cast<uint32_t>(wg * D) : 0u);
         const float sl2 = p.scale_log2;
         const bool pos_scale = sl2 > 0.0f;
-        float m_ref = -INFINITY;   // reference max, log2 domain
+        float m_ref = -INFINITY;   // reference max of this group's tiles, log2 domain
         float l_sum = 0.0f;        // row sum relative to m_ref
         bool ok = true;
+        const int j0 = DUAL ? wg : 0;
+        const int jstep = DUAL ? 2 : 1;
+        const bool active = DUAL || wg == 0;
+        int seen = 0;              // tiles this group has processed
 #pragma unroll 1
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int j = j0; active && j < n_tiles; j += jstep) {
             ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
@@ -529,7 +553,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                              (pos_scale ? sl2 : 1.0f);
             float factor = 1.0f;
             bool rescale = false;
-            if (j == 0) {
+            if (seen == 0) {
                 m_ref = mx;
             } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
                 const float m_new = fmaxf(m_ref, mx);
@@ -557,26 +581,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l_sum = l_sum * factor + tile_sum;
             if (rescale) {
-                // O may only be touched once PV_{j-1} has completed: S_{j+1} was issued
-                // after it, and for the last tile the MMA thread announces PV_{n-2}.
-                const bool w = (j + 1 < n_tiles)
-                                   ? wait_bar(BAR(BAR_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
-                                   : wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
+                // This group's O may only be touched once its previous PV has completed.
+                // DUAL: that is PV_{j-2}, issued before S_j, which has already completed.
+                // Otherwise PV_{j-1}: S_{j+1} was issued after it, and for the last tile
+                // the MMA thread announces PV_{n-2} on the O barrier.
+                bool w = true;
+                if constexpr (!DUAL) {
+                    w = (j + 1 < n_tiles) ? wait_bar(BAR(BAR_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
+                                          : wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
+                }
                 ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int oc = 0; oc < D / 32; ++oc) {
                     uint32_t o[32];
-                    tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+                    tmem_ld32_wait(tmem + lane_base + o_col + oc * 32, o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                    tmem_st32(tmem + lane_base + O_COL + oc * 32, o);
+                    tmem_st32(tmem + lane_base + o_col + oc * 32, o);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(BAR(BAR_P + (j & 1)));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(BAR_P + (j & 1)));
+            ++seen;
         }
         // ---- epilogue: the O barrier completes once per PV among the last two
         if (ok && n_tiles > 0) {
@@ -585,20 +615,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }
-        const int row = q0 + tid;
+        // combine the groups' partial results: m = max_w m_w, f_w = 2^(m_w - m),
+        // l = sum_w l_w f_w, O = sum_w O_w f_w / l (a group with no tile has l_w = 0).
+        float f_own = 1.0f, f_other = 0.0f, m_row = m_ref, l_row = l_sum;
+        bool other_has = false;
+        if constexpr (DUAL) {
+            float* xch = reinterpret_cast<float*>(smem + C::Q_BYTES + C::NSLOTS * C::SLOT + 1024);  // [2][2][128]
+            xch[(wg * 2 + 0) * 128 + r] = m_ref;
+            xch[(wg * 2 + 1) * 128 + r] = l_sum;
+            named_barrier_sync(9, 256);
+            const float m_o = xch[((wg ^ 1) * 2 + 0) * 128 + r];
+            const float l_o = xch[((wg ^ 1) * 2 + 1) * 128 + r];
+            const bool own_has = l_sum > 0.0f;
+            other_has = l_o > 0.0f;
+            m_row = own_has ? (other_has ? fmaxf(m_ref, m_o) : m_ref) : m_o;
+            f_own = own_has ? fast_exp2(m_ref - m_row) : 0.0f;
+            f_other = other_has ? fast_exp2(m_o - m_row) : 0.0f;
+            l_row = l_sum * f_own + l_o * f_other;
+        }
+        const int row = q0 + r;
         const bool in_range = row < p.Tq;
         const bool have = n_tiles > 0;
-        const float inv_l = have ? 1.0f / l_sum : 0.0f;
-        const float lse_val = have ? (m_ref + log2f(l_sum)) * LN2 : -INFINITY;
+        const float inv_l = have ? 1.0f / l_row : 0.0f;
+        const float lse_val = have ? (m_row + log2f(l_row)) * LN2 : -INFINITY;
         const long long BH = static_cast<long long>(p.B) * p.H;
+        const bool own_has_o = DUAL ? (have && l_sum > 0.0f) : have;
+        const uint32_t o_col_other = O_COL + static_cast<uint32_t>((wg ^ 1) * D);
+        // DUAL: group w writes the 32-column chunks oc = w (mod 2); otherwise group 0 writes all
 #pragma unroll 1
-        for (int oc = 0; oc < D / 32; ++oc) {
+        for (int oc = DUAL ? wg : 0; active && oc < D / 32; oc += DUAL ? 2 : 1) {
             uint32_t o[32];
-            if (have) {
-                tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+            if (own_has_o) {
+                tmem_ld32_wait(tmem + lane_base + (DUAL ? O_COL + static_cast<uint32_t>(wg * D) : O_COL) + oc * 32, o);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_own);
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            if (DUAL && other_has) {
+                uint32_t o2[32];
+                tmem_ld32_wait(tmem + lane_base + o_col_other + oc * 32, o2);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[e] = __float_as_uint(fmaf(__uint_as_float(o2[e]), f_other, __uint_as_float(o[e])));
             }
             if (!in_range) continue;
             if constexpr (SPLIT) {
@@ -622,7 +682,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
         }
-        if (in_range) {
+        if (in_range && wg == 0) {
             if constexpr (SPLIT) {
                 p.part_lse[(static_cast<long long>(split) * BH + bh) * p.Tq + row] = lse_val;
             } else if (p.lse != nullptr) {
@@ -633,7 +693,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -796,7 +856,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, Params prm, 
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
-    kern<<<static_cast<unsigned>(grid), attn::NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+    kern<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     return ATTN_OK;
 }

@@ -162,6 +162,11 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 }
 // All threads of every CTA in the cluster; release/acquire orders shared-memory state
 // (barrier initialisation, TMEM address) across the pair.
+// Named barrier `id` over `nthreads` threads (whole warps); id 0 is __syncthreads'.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
