@@ -72,9 +72,11 @@ struct Cfg {
     static constexpr int KCH = NBLK;                  // K tile: one chunk per column block
     static constexpr int VCH = NBLK;                  // V tile: chunks of V_ROWS key rows
     static constexpr int V_ROWS = BN / VCH;
-    // Head dims whose two O accumulators fit in TMEM beside the two S buffers run two
-    // softmax warpgroups (even and odd key tiles); larger ones run one.
-    static constexpr bool DUAL = O_COL + 2 * D <= TMEM_COLS;
+    // Head dims whose two O accumulators and two P buffers fit in TMEM beside the two S
+    // buffers run two softmax warpgroups (even and odd key tiles) with P kept apart from
+    // S; larger ones run one warpgroup with P stored over S.
+    static constexpr bool DUAL = O_COL + 2 * D + BN <= TMEM_COLS;
+    static constexpr uint32_t P_COL = O_COL + 2 * D;    // DUAL: P_w at P_COL + w * BN/2
     static constexpr int SM_WARPS = DUAL ? 8 : 4;
     static constexpr int WARP_PROD = SM_WARPS;          // TMA producer
     static constexpr int WARP_MMA = SM_WARPS + 1;       // MMA issuer, TMEM owner
@@ -102,9 +104,11 @@ enum : int {
     BAR_EMPTY = 17,     // [16] ring group consumed (tcgen05.commit)
     BAR_S = 33,         // [2] S_j ready in TMEM buffer j&1
     BAR_P = 35,         // [2] P_j stored over S_j (one arrival per softmax warp of its group)
-    BAR_O = 37,         // PV complete, announced for the last two tiles only
+    BAR_PVD = 37,       // [2] PV into accumulator O_w complete (one phase per PV)
     BAR_DRAIN = 39,
-    NUM_BARS = 40
+    BAR_SC = 40,        // [2] two-group mode: S_j read out of TMEM buffer j&1 (one arrival per warp)
+    BAR_OFIN = 42,      // the last PV complete (completes once; its commit covers every MMA)
+    NUM_BARS = 43
 };
 
 struct Params {
@@ -247,8 +251,12 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             mbar_init(BAR(BAR_S + i), 1);
             mbar_init(BAR(BAR_P + i), 4);
         }
-        mbar_init(BAR(BAR_O), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(BAR_PVD + i), 1);
+            mbar_init(BAR(BAR_SC + i), 4);
+        }
         mbar_init(BAR(BAR_DRAIN), 1);
+        mbar_init(BAR(BAR_OFIN), 1);
         *abort_flag = 0;
         *ready_seq = 0u;
         fence_mbar_init();
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     if (warp == C::WARP_PROD) {
         // ================================================================ producer
         // Loads go out in the order the MMA thread consumes them: K_0, K_1, then
-        // V_j, K_{j+2} for every tile j.  Each tile half is GRP-chunk groups; one ring
+        // V_j, K_{j+2} for every tile j (two-group mode: K_2, then K_{j+3}, V_j).  Each tile half is GRP-chunk groups; one ring
         // group (GRP consecutive 16 KB slots) has one full and one empty barrier.
         if (lane == 0 && n_tiles > 0) {
             tma_prefetch_map(&tm_q);
@@ -331,10 +339,20 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             };
             load_k(0);
             if (n_tiles > 1) load_k(1);
+            if constexpr (C::DUAL) {
+                // S runs three tiles ahead of PV: K_2, then K_{j+3}, V_j per tile j
+                if (n_tiles > 2) load_k(2);
 #pragma unroll 1
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                load_v(j);
-                if (j + 2 < n_tiles) load_k(j + 2);
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    if (j + 3 < n_tiles) load_k(j + 3);
+                    load_v(j);
+                }
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    load_v(j);
+                    if (j + 2 < n_tiles) load_k(j + 2);
+                }
             }
             if (!ok) {
                 // Drain: every copy issued must land before this CTA's memory is reused.
@@ -408,8 +426,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 // Every 16-key step is issued, partial last tile included: its masked
                 // columns hold P = 0 against value rows that are valid keys of earlier
                 // tiles (or zero fill), never padding.
-                // Two accumulators (DUAL): PV_j adds into O_{j&1}; each starts fresh.
-                const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+                // Two-group mode: PV_j reads P_{j&1} and adds into O_{j&1}; each starts fresh.
+                const uint32_t p_tmem = C::DUAL ? tmem + C::P_COL + static_cast<uint32_t>(j & 1) * (BN / 2)
+                                                : tmem + static_cast<uint32_t>(j & 1) * BN;
                 const uint32_t o_tmem = tmem + O_COL + (C::DUAL ? static_cast<uint32_t>((j & 1) * D) : 0u);
                 const uint32_t acc0 = (j < (C::DUAL ? 2 : 1)) ? 0u : 1u;
 #pragma unroll
@@ -428,10 +447,10 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 }
 #pragma unroll
                 for (int g = 0; g < VG; ++g) tc_commit(BAR(BAR_EMPTY + ring(g)));
-                // O is announced only after the last two PV steps: the softmax rescale of
-                // the last tile and the epilogue are its only readers (earlier rescales
-                // learn that PV_{j-1} is done from S_{j+1}, issued after it).
-                if (j >= n_tiles - 2) tc_commit(BAR(BAR_O));
+                // One phase per PV on the accumulator's barrier: the softmax group waits
+                // it before rescaling O or reusing the P buffer, the epilogue before reading.
+                tc_commit(BAR(BAR_PVD + (C::DUAL ? (j & 1) : 0)));
+                if (j == n_tiles - 1) tc_commit(BAR(BAR_OFIN));
                 advance(VG);
             };
             if (ok) ok = next_event();
@@ -446,17 +465,42 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     issue_s(1);
                 }
             }
+            if constexpr (C::DUAL) {
+                // P has its own buffers, so S_{j+2} may overwrite S_j as soon as the group
+                // has read it out: S runs ahead of PV (S_2, then S_{j+3} before PV_j).
+                if (ok && n_tiles > 2) {
+                    ok = next_event();   // S_0 read out and K_2 landed
+                    if (ok) {
+                        tc_fence_after();
+                        issue_s(2);
+                    }
+                }
 #pragma unroll 1
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                ok = next_event();   // P_j stored and V_j landed
-                if (!ok) break;
-                tc_fence_after();
-                issue_pv(j);
-                if (j + 2 < n_tiles) {
-                    ok = next_event();   // K_{j+2} landed
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    if (j + 3 < n_tiles) {
+                        ok = next_event();   // S_{j+1} read out and K_{j+3} landed
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(j + 3);
+                    }
+                    ok = next_event();   // P_j stored and V_j landed
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(j + 2);
+                    issue_pv(j);
+                }
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    ok = next_event();   // P_j stored and V_j landed
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(j);
+                    if (j + 2 < n_tiles) {
+                        ok = next_event();   // K_{j+2} landed
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(j + 2);
+                    }
                 }
             }
             // Drain: every MMA issued completes before TMEM is released.
@@ -469,6 +513,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         // Waits on the ring groups and P barriers in the MMA thread's consumption order
         // and publishes one completed event per MMA batch with a release store: K_0,
         // K_1, then per tile j "P_j + V_j" and "K_{j+2}"; the MMA thread acquires it.
+        // Two-group mode: K_0, K_1, "S_0 read + K_2", then per tile j "S_{j+1} read +
+        // K_{j+3}" and "P_j + V_j".
         if (lane == 0 && n_tiles > 0) {
             int gi = 0;
             uint32_t phase = 0, seq = 0;
@@ -489,23 +535,43 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             };
             relay_s();
             if (n_tiles > 1) relay_s();
+            if constexpr (C::DUAL) {
+                auto s_read = [&](int t) {
+                    ok = ok && wait_bar(BAR(BAR_SC + (t & 1)), (t >> 1) & 1, abort_flag, wlim);
+                };
+                if (n_tiles > 2) {
+                    s_read(0);
+                    relay_s();
+                }
 #pragma unroll 1
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
-                for (int g = 0; g < C::VCH / C::GRP; ++g) group();
-                publish();
-                if (j + 2 < n_tiles) relay_s();
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    if (j + 3 < n_tiles) {
+                        s_read(j + 1);
+                        relay_s();
+                    }
+                    ok = ok && wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();
+                    publish();
+                }
+            } else {
+#pragma unroll 1
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();
+                    publish();
+                    if (j + 2 < n_tiles) relay_s();
+                }
             }
         }
         __syncwarp();
     } else {
         // ================================================================ softmax
         // Thread t of warpgroup w (warps 4w .. 4w+3) owns query row r = t % 128 (TMEM lane r).
-        // Head dims up to 64 (DUAL): warpgroup w takes the key tiles j = w (mod 2) with its
-        // own running max, row sum and O accumulator (TMEM columns O_COL + w*D), so one
-        // group's max phase overlaps the other's exponentials; the two partial results are
-        // combined exactly at the end (the log-sum-exp rule of split-KV).  Head dim 256
-        // (test hook only) keeps one accumulator and warpgroup 0 takes every tile.
+        // Two-group mode (head dims up to 64): warpgroup w takes the key tiles j = w (mod 2)
+        // with its own running max, row sum, O accumulator O_w and P buffer P_w, so one
+        // group's exponentials overlap the other's MMA round trip; the two partial results
+        // are combined exactly at the end (the log-sum-exp rule of split-KV).  Otherwise one
+        // warpgroup takes every tile and stores P over S.
         constexpr bool DUAL = C::DUAL;
         const int wg = warp >> 2;
         const int r = tid & 127;
@@ -518,16 +584,22 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         bool ok = true;
         const int j0 = DUAL ? wg : 0;
         const int jstep = DUAL ? 2 : 1;
-        const bool active = DUAL || wg == 0;
         int seen = 0;              // tiles this group has processed
+        // One arrival per warp once its tcgen05 accesses are complete.
+        auto warp_arrive = [&](uint32_t bar) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
 #pragma unroll 1
-        for (int j = j0; active && j < n_tiles; j += jstep) {
+        for (int j = j0; j < n_tiles; j += jstep) {
             ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
             uint32_t raw[BN];
             tmem_ld128_wait(s_addr, raw);
+            if constexpr (DUAL) warp_arrive(BAR(BAR_SC + (j & 1)));   // S buffer free for S_{j+2}
             float x[BN];
             const int lo = (j == n_tiles - 1) ? last_lo : 0;   // columns [0, lo) are not this tile's keys
             if (lo > 0) {
@@ -566,33 +638,33 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             float sp[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
+            uint32_t pk[BN / 2];
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
                     const float p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
                     sp[e & 7] += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    pk[cc * 16 + e] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(s_addr + cc * 16, pk);
+                if constexpr (!DUAL) tmem_st16_at(s_addr + cc * 16, &pk[cc * 16]);   // P over S_j
             }
             const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l_sum = l_sum * factor + tile_sum;
-            if (rescale) {
-                // This group's O may only be touched once its previous PV has completed.
-                // DUAL: that is PV_{j-2}, issued before S_j, which has already completed.
-                // Otherwise PV_{j-1}: S_{j+1} was issued after it, and for the last tile
-                // the MMA thread announces PV_{n-2} on the O barrier.
-                bool w = true;
-                if constexpr (!DUAL) {
-                    w = (j + 1 < n_tiles) ? wait_bar(BAR(BAR_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
-                                          : wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
-                }
-                ok = __all_sync(0xffffffffu, w);
+            // This group's previous PV (PV_{j-2} in two-group mode, else PV_{j-1}) must be
+            // complete before O is rescaled, and (two-group mode) before P_w is rewritten.
+            // The parity wait is unambiguous: the barrier has passed the phase before
+            // (two-group mode: this group waited for it on its previous tile; one group:
+            // S_j, issued after PV_{j-2}, is complete) and cannot pass the one after, whose
+            // PV needs this tile's P.
+            if (seen > 0 && (DUAL || rescale)) {
+                ok = __all_sync(0xffffffffu,
+                                wait_bar(BAR(BAR_PVD + (DUAL ? (j & 1) : 0)), (seen - 1) & 1, abort_flag, wlim));
                 if (!ok) break;
                 tc_fence_after();
+            }
+            if (rescale) {
 #pragma unroll 1
                 for (int oc = 0; oc < D / 32; ++oc) {
                     uint32_t o[32];
@@ -602,17 +674,20 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     tmem_st32(tmem + lane_base + o_col + oc * 32, o);
                 }
             }
+            if constexpr (DUAL) {
+                const uint32_t p_addr = tmem + lane_base + C::P_COL + static_cast<uint32_t>(j & 1) * (BN / 2);
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) tmem_st16_at(p_addr + cc * 16, &pk[cc * 16]);
+            }
             tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(BAR_P + (j & 1)));
+            warp_arrive(BAR(BAR_P + (j & 1)));
             ++seen;
         }
-        // ---- epilogue: the O barrier completes once per PV among the last two
+        // ---- epilogue: the last PV's barrier completes once, after every MMA.  (A parity
+        // wait names a phase only while the barrier is at most one phase from it, which
+        // the per-PV barriers do not promise here.)
         if (ok && n_tiles > 0) {
-            bool w = wait_bar(BAR(BAR_O), 0, abort_flag, wlim);
-            if (n_tiles > 1) w = w && wait_bar(BAR(BAR_O), 1, abort_flag, wlim);
-            ok = __all_sync(0xffffffffu, w);
+            ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_OFIN), 0, abort_flag, wlim));
             tc_fence_after();
         }
         // combine the groups' partial results: m = max_w m_w, f_w = 2^(m_w - m),
@@ -643,7 +718,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         const uint32_t o_col_other = O_COL + static_cast<uint32_t>((wg ^ 1) * D);
         // DUAL: group w writes the 32-column chunks oc = w (mod 2); otherwise group 0 writes all
 #pragma unroll 1
-        for (int oc = DUAL ? wg : 0; active && oc < D / 32; oc += DUAL ? 2 : 1) {
+        for (int oc = DUAL ? wg : 0; oc < D / 32; oc += DUAL ? 2 : 1) {
             uint32_t o[32];
             if (own_has_o) {
                 tmem_ld32_wait(tmem + lane_base + (DUAL ? O_COL + static_cast<uint32_t>(wg * D) : O_COL) + oc * 32, o);

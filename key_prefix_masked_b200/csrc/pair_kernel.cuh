@@ -46,10 +46,11 @@ enum : int {
     PB_FULL = 1,     // [8] slot filled by both CTAs' copies (leader)
     PB_EMPTY = 9,    // [8] slot consumed (multicast commit, both CTAs)
     PB_S = 17,       // [2] S_j ready (multicast commit, both CTAs)
-    PB_O = 19,       // PV of the last two tiles complete (multicast commit, both CTAs)
+    PB_OLAST = 19,   // PV_{n-1} complete (multicast commit, both CTAs; completes once)
     PB_DRAIN = 20,   // leader only
     PB_P = 21,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
-    PB_NUM = 23
+    PB_OPREV = 23,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
+    PB_NUM = 24
 };
 
 template <bool SPLIT>
@@ -111,7 +112,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         mbar_init(PBAR(PB_S + 0), 1);
         mbar_init(PBAR(PB_S + 1), 1);
-        mbar_init(PBAR(PB_O), 1);
+        mbar_init(PBAR(PB_OLAST), 1);
+        mbar_init(PBAR(PB_OPREV), 1);
         mbar_init(PBAR(PB_DRAIN), 1);
         mbar_init(PBAR(PB_P + 0), 8);
         mbar_init(PBAR(PB_P + 1), 8);
@@ -278,7 +280,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                                 vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV,
                                 (j == 0 && kb == 0) ? 0u : 1u);
                 tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
-                if (j >= n_tiles - 2) tc_commit_pair(PBAR(PB_O), 0x3);
+                // Each O barrier completes exactly once, so a parity-0 wait on it cannot
+                // be confused by a later phase.
+                if (j == n_tiles - 2) tc_commit_pair(PBAR(PB_OPREV), 0x3);
+                if (j == n_tiles - 1) tc_commit_pair(PBAR(PB_OLAST), 0x3);
                 next_slot();
             };
             if (ok) issue_s(0);
@@ -360,10 +365,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             l_sum = l_sum * factor + tile_sum;
             if (rescale) {
                 // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last tile
-                // the leader announces PV_{n-2} on the O barrier.
+                // the leader announces PV_{n-2} on its own barrier.
                 const bool w = (j + 1 < n_tiles)
                                    ? wait_bar(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
-                                   : wait_bar(PBAR(PB_O), 0, abort_flag, wlim);
+                                   : wait_bar(PBAR(PB_OPREV), 0, abort_flag, wlim);
                 ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
                 tc_fence_after();
@@ -383,8 +388,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         // ---- epilogue
         if (ok && n_tiles > 0) {
-            bool w = wait_bar(PBAR(PB_O), 0, abort_flag, wlim);
-            if (n_tiles > 1) w = w && wait_bar(PBAR(PB_O), 1, abort_flag, wlim);
+            // PV_{n-1}'s commit tracks every earlier MMA of the leader's thread as well
+            const bool w = wait_bar(PBAR(PB_OLAST), 0, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }
