@@ -55,6 +55,7 @@ constexpr int SMEM_LIMIT = 232448;    // 227 KB opt-in dynamic shared memory per
 constexpr uint32_t TMEM_COLS = 512;   // S0 [0,128) S1 [128,256) O [256, 256+D)
 constexpr uint32_t O_COL = 256;
 constexpr float RESCALE_LOG2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr uint32_t XCH_ID = 9;     // named barrier: the two softmax groups' epilogue exchange
 constexpr float LN2 = 0.69314718055994530942f;
 constexpr float LOG2E = 1.44269504088896340736f;
 
@@ -108,7 +109,8 @@ enum : int {
     BAR_DRAIN = 39,
     BAR_SC = 40,        // [2] two-group mode: S_j read out of TMEM buffer j&1 (one arrival per warp)
     BAR_OFIN = 42,      // the last PV complete (completes once; its commit covers every MMA)
-    NUM_BARS = 43
+    BAR_TURN = 43,      // [2] two-group mode: group w may run the exponentials of its next tile
+    NUM_BARS = 45
 };
 
 struct Params {
@@ -254,6 +256,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(BAR_PVD + i), 1);
             mbar_init(BAR(BAR_SC + i), 4);
+            mbar_init(BAR(BAR_TURN + i), 4);
         }
         mbar_init(BAR(BAR_DRAIN), 1);
         mbar_init(BAR(BAR_OFIN), 1);
@@ -593,7 +596,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         };
 #pragma unroll 1
         for (int j = j0; j < n_tiles; j += jstep) {
-            ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
             const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
@@ -635,6 +638,17 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             }
             const float mul = pos_scale ? sl2 : 1.0f;
             const float neg_m = -m_ref;
+            if constexpr (DUAL) {
+                // The groups take turns at the exponentials in tile order, so one group's
+                // MUFU-bound phase overlaps the other's loads, max and MMA round trip
+                // instead of both contending for the MUFU at once.  Group w waits on
+                // TURN_w; the group that ran tile j - 1 arrives on it after its exponentials.
+                if (j >= 1) {
+                    ok = __all_sync(0xffffffffu,
+                                    wait_bar(BAR(BAR_TURN + (j & 1)), ((j - 1) >> 1) & 1, abort_flag, wlim));
+                    if (!ok) break;
+                }
+            }
             float sp[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
@@ -649,6 +663,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     pk[cc * 16 + e] = pack_bf16x2(p0, p1);
                 }
                 if constexpr (!DUAL) tmem_st16_at(s_addr + cc * 16, &pk[cc * 16]);   // P over S_j
+            }
+            if constexpr (DUAL) {
+                if (j + 1 < n_tiles) warp_arrive(BAR(BAR_TURN + ((j + 1) & 1)));
             }
             const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l_sum = l_sum * factor + tile_sum;
@@ -698,7 +715,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             float* xch = reinterpret_cast<float*>(smem + C::Q_BYTES + C::NSLOTS * C::SLOT + 1024);  // [2][2][128]
             xch[(wg * 2 + 0) * 128 + r] = m_ref;
             xch[(wg * 2 + 1) * 128 + r] = l_sum;
-            named_barrier_sync(9, 256);
+            named_barrier_sync(XCH_ID, 256);
             const float m_o = xch[((wg ^ 1) * 2 + 0) * 128 + r];
             const float l_o = xch[((wg ^ 1) * 2 + 1) * 128 + r];
             const bool own_has = l_sum > 0.0f;
