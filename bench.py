@@ -9,7 +9,10 @@ partial launch plus the LSE combine.  FLOPs counted = sum_b 4*H*Tq*kv_len[b]*D.
 
 The default workload is the in-context-learning shape: B=1, H=8, D=256, 110000 queries
 against 100000 valid keys in a 100352-row padded key buffer.  Its inputs (1.27 GB) are
-larger than the 126 MB L2, so no flush is needed between steps.
+larger than the 126 MB L2, so no flush is needed between steps.  A workload whose
+q, k and v together are smaller than twice the L2 (the D=64 shapes) gets a 252 MB buffer
+written before every timed step, outside that step's CUDA events; its value then comes
+from the per-step events.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of the
 workload (weak scaling, no collective on the data path); the step time is the max over
@@ -41,6 +44,7 @@ import synth  # noqa: E402
 METRIC = "attention fwd TFLOP/s (valid keys only) and % of BF16 tensor peak on one B200"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
 
 
 def load_peaks():
@@ -204,6 +208,8 @@ def run_ours(args, rank, world):
         raise RuntimeError(f"device status after warm-up: {kp.status_string(st)}")
 
     # ---- device-timed region: inputs resident in HBM
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     k_ev = []   # per-launch events of the dominant kernel (the attention launch)
@@ -214,6 +220,8 @@ def run_ours(args, rank, world):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()   # evict the inputs from L2 (outside the step's events)
             ev[i][0].record(stream)
             if splits:
                 a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -232,8 +240,8 @@ def run_ours(args, rank, world):
     st = kp.device_status()
     if st != kp.ATTN_OK:
         raise RuntimeError(f"device status after timing: {kp.status_string(st)}")
-    total_ms = t0.elapsed_time(t1)
     step_ms = [a.elapsed_time(b_) for a, b_ in ev]
+    total_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
     kern_ms = ([a.elapsed_time(b_) for a, b_ in k_ev] if k_ev else step_ms)
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
@@ -271,7 +279,9 @@ def run_ours(args, rank, world):
         "data": "synthetic (seeded N(0,std^2) bf16 q/k/v, NaN in padded key slots)",
         "config": {**w.describe(), "kv_len": case["kv_len_list"] if len(case["kv_len_list"]) <= 8
                    else "ragged", "scale": scale, "flops_per_step": flops,
-                   "l2": "inputs larger than the 126 MB L2; no flush",
+                   "l2": ("inputs larger than the 126 MB L2; no flush" if flush is None else
+                          "inputs smaller than 2x L2: a 252 MB buffer written before each step, "
+                          "outside the step events; value from per-step events"),
                    "parallelism": f"replicas x{world}"},
         "impl": "ours",
         "e2e": e2e,
