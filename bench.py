@@ -262,12 +262,16 @@ def run_ours(args, rank, world):
     kernel_tag = "attn_fwd_pair" if w.D == 256 else f"attn_fwd_d{w.D}"
     kernel_name = (f"attn_fwd_pair_kernel<{int(bool(splits))}>" if w.D == 256
                    else f"attn_fwd_kernel<{w.D},{int(bool(splits))}>")
-    peak_key = "bf16_tflops_sustained"
+    # A kernel that runs long enough to draw the power cap is compared with the sustained
+    # cuBLAS figure; a short one (the D=64 shapes, ~1 ms steps) with the burst figure.
+    long_run = total_ms >= 1000.0 or "sw_power_cap" in (clocks.get("reasons") or [])
+    peak_key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
     peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
     roofline = {
         "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
         "frac": round(achieved / peak, 4),
-        "peak_source": f"{peaks_src} {peak_key} (kernel timed inside a seconds-long back-to-back loop)",
+        "peak_source": f"{peaks_src} {peak_key} " + ("(kernel under the power cap in a long back-to-back loop)"
+                                                      if long_run else "(short kernel, no power cap: burst figure)"),
         "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
         "traffic": traffic_from_profile(args.workload, kernel_tag),
         "kernel": kernel_name,
