@@ -5,7 +5,8 @@
 One step = one pass of the hot path over one batch of the workload, inputs resident in
 HBM: for the single-pass workloads one attn_prefix_fwd launch (key-range selection,
 TMA staging, QK^T, prefix mask, online softmax, PV, epilogue); for `splitkv` the split
-partial launch plus the LSE combine.  FLOPs counted = sum_b 4*H*Tq*kv_len[b]*D.
+partial launch plus the LSE combine launch (`--split-mode fused`: one launch whose last
+chunk per query tile runs the combine, attn_prefix_fwd_split_fused).  FLOPs counted = sum_b 4*H*Tq*kv_len[b]*D.
 
 The default workload is the in-context-learning shape: B=1, H=8, D=256, 110000 queries
 against 100000 valid keys in a 100352-row padded key buffer.  Its inputs (1.27 GB) are
@@ -186,20 +187,30 @@ def run_ours(args, rank, world):
     splits = w.num_splits if w.num_splits > 1 else 0
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=dev)
-    ws = None
-    if splits:
-        ws = (torch.empty((splits, w.B, w.H, w.Tq, w.D), dtype=torch.float32, device=dev),
+    fused = bool(splits) and args.split_mode == "fused"
+    ws = kp.fused_workspace(splits, w.B, w.H, w.Tq, w.D, dev) if fused else None
+    parts = ((torch.empty((splits, w.B, w.H, w.Tq, w.D), dtype=torch.float32, device=dev),
               torch.empty((splits, w.B, w.H, w.Tq), dtype=torch.float32, device=dev))
+             if splits and not fused else None)
     stream = torch.cuda.current_stream(dev)
+    k_ev = []   # separate split mode: events around the split launch (the dominant kernel)
 
-    def step(qq, kk, vv, kvl):
-        if splits:
-            kp.attn_prefix_fwd_split(qq, kk, vv, kvl, splits, scale, *ws)
-            kp.attn_lse_combine(ws[0], ws[1], out=out, lse=lse)
+    def step(qq, kk, vv, kvl, timed=False):
+        if fused:
+            kp.attn_prefix_fwd_split_fused(qq, kk, vv, kvl, splits, scale, workspace=ws, out=out, lse=lse)
+        elif splits:
+            if timed:
+                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            kp.attn_prefix_fwd_split(qq, kk, vv, kvl, splits, scale, *parts)
+            if timed:
+                b_.record(stream)
+                k_ev.append((a, b_))
+            kp.attn_lse_combine(parts[0], parts[1], out=out, lse=lse)
         else:
             kp.attn_prefix_fwd(qq, kk, vv, kvl, scale, out=out, lse=lse)
 
-    launches_per_step = 2 if splits else 1
+    launches_per_step = 2 if (splits and not fused) else 1
     for _ in range(args.warmup):
         step(q, k, v, kv)
     torch.cuda.synchronize()
@@ -212,7 +223,6 @@ def run_ours(args, rank, world):
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    k_ev = []   # per-launch events of the dominant kernel (the attention launch)
     with ClockMonitor(torch.cuda.current_device()) as mon:
         barrier(world)
         torch.cuda.synchronize()
@@ -223,15 +233,7 @@ def run_ours(args, rank, world):
             if flush is not None:
                 flush.zero_()   # evict the inputs from L2 (outside the step's events)
             ev[i][0].record(stream)
-            if splits:
-                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                kp.attn_prefix_fwd_split(q, k, v, kv, splits, scale, *ws)
-                b_.record(stream)
-                k_ev.append((a, b_))
-                kp.attn_lse_combine(ws[0], ws[1], out=out, lse=lse)
-            else:
-                kp.attn_prefix_fwd(q, k, v, kv, scale, out=out, lse=lse)
+            step(q, k, v, kv, timed=True)
             ev[i][1].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
@@ -242,13 +244,13 @@ def run_ours(args, rank, world):
         raise RuntimeError(f"device status after timing: {kp.status_string(st)}")
     step_ms = [a.elapsed_time(b_) for a, b_ in ev]
     total_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
-    kern_ms = ([a.elapsed_time(b_) for a, b_ in k_ev] if k_ev else step_ms)
+    kern_ms = [a.elapsed_time(b_) for a, b_ in k_ev] if k_ev else step_ms
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(flops, world, ms_per_step)
 
     # ---- end-to-end: pinned host buffers, copies inside the timed region
-    e2e = run_e2e(kp, w, case, scale, splits, args, world)
+    e2e = run_e2e(kp, w, case, scale, splits, fused, args, world)
 
     # ---- quick correctness check on a few sampled rows (outside every timed region)
     verified = None
@@ -286,7 +288,8 @@ def run_ours(args, rank, world):
                    "l2": ("inputs larger than the 126 MB L2; no flush" if flush is None else
                           "inputs smaller than 2x L2: a 252 MB buffer written before each step, "
                           "outside the step events; value from per-step events"),
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   **({"split_mode": args.split_mode} if splits else {})},
         "impl": "ours",
         "e2e": e2e,
         "roofline": roofline,
@@ -301,7 +304,7 @@ def run_ours(args, rank, world):
     return rec
 
 
-def run_e2e(kp, w, case, scale, splits, args, world):
+def run_e2e(kp, w, case, scale, splits, fused, args, world):
     """Same metric through the public call with host buffers: every step copies that
     step's inputs host->device from pinned memory and reads the result back."""
     dev = case["q"].device
@@ -314,10 +317,10 @@ def run_e2e(kp, w, case, scale, splits, args, world):
     dq, dk, dv, dkv = (torch.empty_like(case[n]) for n in ("q", "k", "v", "kv_len"))
     dout = torch.empty_like(case["q"])
     dlse = torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=dev)
-    ws = None
-    if splits:
-        ws = (torch.empty((splits, w.B, w.H, w.Tq, w.D), dtype=torch.float32, device=dev),
+    ws = kp.fused_workspace(splits, w.B, w.H, w.Tq, w.D, dev) if fused else None
+    parts = ((torch.empty((splits, w.B, w.H, w.Tq, w.D), dtype=torch.float32, device=dev),
               torch.empty((splits, w.B, w.H, w.Tq), dtype=torch.float32, device=dev))
+             if splits and not fused else None)
     stream = torch.cuda.current_stream(dev)
 
     def one():
@@ -325,9 +328,11 @@ def run_e2e(kp, w, case, scale, splits, args, world):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dkv.copy_(hkv, non_blocking=True)
-        if splits:
-            kp.attn_prefix_fwd_split(dq, dk, dv, dkv, splits, scale, *ws)
-            kp.attn_lse_combine(ws[0], ws[1], out=dout, lse=dlse)
+        if fused:
+            kp.attn_prefix_fwd_split_fused(dq, dk, dv, dkv, splits, scale, workspace=ws, out=dout, lse=dlse)
+        elif splits:
+            kp.attn_prefix_fwd_split(dq, dk, dv, dkv, splits, scale, *parts)
+            kp.attn_lse_combine(parts[0], parts[1], out=dout, lse=dlse)
         else:
             kp.attn_prefix_fwd(dq, dk, dv, dkv, scale, out=dout, lse=dlse)
         hout.copy_(dout, non_blocking=True)
@@ -453,6 +458,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-verify", dest="verify", action="store_false")
+    ap.add_argument("--split-mode", default="separate", choices=["separate", "fused"],
+                    help="split-KV workloads: the LSE combine as a second launch (faster on B200), "
+                         "or fused into the split launch")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

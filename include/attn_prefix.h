@@ -95,6 +95,31 @@ attn_status attn_lse_combine(const float* part_out, const float* part_lse, int n
                              void* out, float* lse, int B, int H, int Tq, int D,
                              cudaStream_t stream);
 
+/* Split-KV forward with the combine fused into the same launch: the split partials of
+ * attn_prefix_fwd_split, then, inside the kernel, the exact combination of
+ * attn_lse_combine.  The pages combine shard results by log-sum-exp weights so that
+ * only softmax statistics cross ("Add sequence-parallel multi-GPU inference ...",
+ * section "Sequence-parallel inference"); here the last chunk to finish a 128-row
+ * query tile combines that tile, so no second launch re-reads the partials from DRAM.
+ *   workspace: device memory of attn_split_fused_workspace_bytes(num_splits, B, H, Tq, D)
+ *     bytes, 16-byte aligned, owned by the caller: part_out at offset 0, part_lse at
+ *     attn_split_lse_offset, then B*H*ceil(Tq/128) int32 tile counters at
+ *     attn_split_counter_offset.  The counters must be zero before the first call
+ *     (e.g. one cudaMemsetAsync of the workspace); every call that completes leaves them
+ *     zero again, so a workspace is reused without clearing.  After a call that raised
+ *     a device error flag (attn_get_device_status != ATTN_OK), zero them again.  Calls
+ *     sharing one workspace must not overlap on the GPU.
+ *   out: bf16 [B,H,Tq,D]; lse: fp32 [B,H,Tq] or NULL.  Same result, bit for bit, as
+ *   attn_prefix_fwd_split followed by attn_lse_combine.  Other arguments and checks as
+ *   attn_prefix_fwd_split. */
+size_t attn_split_counter_offset(int num_splits, int B, int H, int Tq, int D);
+size_t attn_split_fused_workspace_bytes(int num_splits, int B, int H, int Tq, int D);
+attn_status attn_prefix_fwd_split_fused(const void* q, const void* k, const void* v,
+                                        const int32_t* kv_len, int num_splits, void* workspace,
+                                        void* out, float* lse,
+                                        int B, int H, int Tq, int Tk, int D, float scale,
+                                        cudaStream_t stream);
+
 /* Split-KV forward that allocates nothing, for callers that cannot call cudaMalloc.
  * The pages have no counterpart to this entry point: it exists for the integration
  * side, not for the method.  Some callers only ever receive device memory for their

@@ -1,7 +1,8 @@
 """B200-native (sm_100a) prefix-masked attention forward.
 
     out, lse = attn_prefix_fwd(q, k, v, kv_len)          # single pass
-    out, lse = attn_prefix_fwd_splitkv(q, k, v, kv_len, num_splits=64)
+    out, lse = attn_prefix_fwd_splitkv(q, k, v, kv_len, num_splits=64)      # split + combine
+    out, lse = attn_prefix_fwd_split_fused(q, k, v, kv_len, num_splits=64)  # one launch
 
 q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 256}; kv_len:
 int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never take part).
@@ -23,6 +24,8 @@ from ._binding import (  # noqa: F401
     fwd as attn_prefix_fwd,
     fwd_split as attn_prefix_fwd_split,
     fwd_splitkv as attn_prefix_fwd_splitkv,
+    fwd_split_fused as attn_prefix_fwd_split_fused,
+    fused_workspace,
     lib,
     lse_combine as attn_lse_combine,
     set_debug_flags,

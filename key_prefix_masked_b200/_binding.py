@@ -37,6 +37,9 @@ _SIGNATURES = {
     "attn_split_lse_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_prefix_fwd_split": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_lse_combine": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_split_counter_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_split_fused_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "attn_prefix_fwd_split_fused": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_prefix_fwd_splitkv_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
@@ -166,6 +169,41 @@ def fwd_splitkv(q, k, v, kv_len, num_splits, scale=None, workspace=None):
     part_out, part_lse = fwd_split(q, k, v, kv_len, num_splits, scale,
                                    *(workspace if workspace is not None else (None, None)))
     return lse_combine(part_out, part_lse)
+
+
+def fused_workspace(num_splits, B, H, Tq, D, device):
+    """A zeroed workspace for fwd_split_fused (partials + tile counters), as uint8."""
+    n = int(lib().attn_split_fused_workspace_bytes(int(num_splits), int(B), int(H), int(Tq), int(D)))
+    if n == 0:
+        raise ValueError("invalid split shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def fwd_split_fused(q, k, v, kv_len, num_splits, scale=None, workspace=None, out=None, lse=None,
+                    need_lse=True):
+    """Split-KV forward with the combine fused into the launch (attn_prefix_fwd_split_fused).
+
+    `workspace` (from fused_workspace, reusable: the kernel leaves its counters zero) is
+    allocated and zeroed here when not given.  Returns (out bf16, lse fp32)."""
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len)
+    C = int(num_splits)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if workspace is None:
+        workspace = fused_workspace(C, B, H, Tq, D, q.device)
+    need = int(lib().attn_split_fused_workspace_bytes(C, B, H, Tq, D))
+    if (not workspace.is_cuda or workspace.device != q.device or not workspace.is_contiguous()
+            or workspace.numel() * workspace.element_size() < need):
+        raise ValueError(f"workspace must be a contiguous CUDA buffer of at least {need} bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib().attn_prefix_fwd_split_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), C, _ptr(workspace),
+                                               _ptr(out), _ptr(lse), B, H, Tq, Tk, D, scale,
+                                               _stream_ptr(q.device))
+    _check(st, "attn_prefix_fwd_split_fused")
+    return out, lse
 
 
 def device_status(device=None) -> int:

@@ -115,10 +115,11 @@ enum : int {
 
 struct Params {
     const int32_t* kv_len;
-    __nv_bfloat16* out;   // single pass: bf16 [B,H,Tq,D]
-    float* lse;           // single pass: fp32 [B,H,Tq] or null
+    __nv_bfloat16* out;   // single pass, or split with fused combine: bf16 [B,H,Tq,D]
+    float* lse;           // single pass, or split with fused combine: fp32 [B,H,Tq] or null
     float* part_out;      // split: fp32 [C,B,H,Tq,D]
     float* part_lse;      // split: fp32 [C,B,H,Tq]
+    int* counters;        // split with fused combine: int32 [B*H*ceil(Tq/128)], else null
     int B, H, Tq, Tk;
     int n_qtiles;
     int num_splits;
@@ -195,6 +196,94 @@ __device__ __noinline__ bool wait_bar_drain_cl(uint32_t bar, uint32_t parity, un
         }
     }
     return true;
+}
+
+// Exact combination of one row's split partials, by one warp (lane = thread % 32):
+//   M = max_c lse_c,  lse = M + ln sum_c exp(lse_c - M),  out = sum_c exp(lse_c - lse) O_c,
+// the log-sum-exp rule of split-KV; a row whose every chunk is empty gives 0 / -inf.
+// Partials are [C][rows][D] and [C][rows].  FRESH: the partials were written by other
+// CTAs of the running kernel, so they are read through L2 (ld.global.cg) instead of the
+// read-only path; the arithmetic, and so the result, is the same either way.
+template <typename T, bool FRESH>
+__device__ __forceinline__ T ld_part(const T* ptr) {
+    if constexpr (FRESH) return __ldcg(ptr);
+    else return __ldg(ptr);
+}
+template <int D, bool FRESH>
+__device__ __forceinline__ void combine_row(const float* __restrict__ part_out, const float* __restrict__ part_lse,
+                                            int C, long long rows, long long row, __nv_bfloat16* __restrict__ out,
+                                            float* __restrict__ lse, int lane) {
+    constexpr int PER = D / 32;
+    float M = -INFINITY;
+    for (int c = lane; c < C; c += 32) M = fmaxf(M, ld_part<float, FRESH>(part_lse + c * rows + row));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    float L = -INFINITY;
+    if (M != -INFINITY) {
+        float s = 0.0f;
+        for (int c = lane; c < C; c += 32) s += expf(ld_part<float, FRESH>(part_lse + c * rows + row) - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        L = M + logf(s);
+        for (int c = 0; c < C; ++c) {
+            const float w = expf(ld_part<float, FRESH>(part_lse + c * rows + row) - L);
+            if (w == 0.0f) continue;   // an empty chunk (lse_c = -inf) adds nothing
+            const float* src = part_out + (static_cast<long long>(c) * rows + row) * D + lane * PER;
+            if constexpr (PER % 4 == 0) {
+#pragma unroll
+                for (int e = 0; e < PER; e += 4) {
+                    const float4 v4 = ld_part<float4, FRESH>(reinterpret_cast<const float4*>(src + e));
+                    acc[e] += w * v4.x;
+                    acc[e + 1] += w * v4.y;
+                    acc[e + 2] += w * v4.z;
+                    acc[e + 3] += w * v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) acc[e] += w * ld_part<float, FRESH>(src + e);
+            }
+        }
+    }
+    __nv_bfloat16* dst = out + row * D + lane * PER;
+    if constexpr (PER == 1) {
+        dst[0] = __float2bfloat16_rn(acc[0]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < PER; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+    }
+    if (lane == 0 && lse != nullptr) lse[row] = L;
+}
+
+// Split-KV with the combine fused in: called by all `nthreads` threads of a CTA (thread
+// index `t`) at its very end, once its partials for query rows [q0, q0 + 128) are stored.  Every CTA of every chunk counts itself in on the tile's counter; the
+// one that completes the count (the last chunk to finish, in whatever order) combines
+// the tile's rows from all chunks' partials into p.out / p.lse and zeroes the counter
+// for the next call.  This is the "only softmax statistics cross" combine of split-KV
+// without a second launch or a second pass over the partials from DRAM.  The count is
+// taken even after an abort, so the counters always return to zero.
+template <int D>
+__device__ __forceinline__ void fused_combine_tail(const Params& p, int bh, int q0, int t, int nthreads,
+                                                   volatile int* flag) {
+    if (q0 >= p.Tq) return;   // a pair's second tile past the last query row: no rows
+    __threadfence();          // this thread's partial stores, visible device-wide
+    __syncthreads();
+    const long long tile = static_cast<long long>(bh) * ((p.Tq + BM - 1) / BM) + q0 / BM;
+    if (t == 0) {
+        const int last = atomicAdd(p.counters + tile, 1) == p.num_splits - 1;
+        if (last) p.counters[tile] = 0;
+        *flag = last;
+    }
+    __syncthreads();
+    if (!*flag) return;
+    __threadfence();          // the other chunks' partials, counted in before the count completed
+    const long long rows = static_cast<long long>(p.B) * p.H * p.Tq;
+    const int nr = min(BM, p.Tq - q0);
+    for (int r = t >> 5; r < nr; r += nthreads >> 5)
+        combine_row<D, true>(p.part_out, p.part_lse, p.num_splits, rows, static_cast<long long>(bh) * p.Tq + q0 + r,
+                             p.out, p.lse, t & 31);
 }
 
 template <int D, bool SPLIT>
@@ -789,62 +878,24 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    if constexpr (SPLIT) {
+        if (p.counters != nullptr)
+            fused_combine_tail<D>(p, bh, q0, tid, C::THREADS, reinterpret_cast<volatile int*>(tmem_holder + 3));
+    }
 #undef BAR
 }
 
 #include "pair_kernel.cuh"
 
-// One warp per output row: lse = M + ln sum_c exp(lse_c - M), out = sum_c exp(lse_c - lse) O_c.
+// One warp per output row (see combine_row).
 template <int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_out,
                                                           const float* __restrict__ part_lse, int C,
                                                           long long rows, __nv_bfloat16* __restrict__ out,
                                                           float* __restrict__ lse) {
-    constexpr int PER = D / 32;
-    const int lane = threadIdx.x & 31;
     const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (row >= rows) return;
-    float M = -INFINITY;
-    for (int c = lane; c < C; c += 32) M = fmaxf(M, __ldg(part_lse + c * rows + row));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-    float L = -INFINITY;
-    if (M != -INFINITY) {
-        float s = 0.0f;
-        for (int c = lane; c < C; c += 32) s += expf(__ldg(part_lse + c * rows + row) - M);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        L = M + logf(s);
-        for (int c = 0; c < C; ++c) {
-            const float w = expf(__ldg(part_lse + c * rows + row) - L);
-            if (w == 0.0f) continue;   // an empty chunk (lse_c = -inf) adds nothing
-            const float* src = part_out + (static_cast<long long>(c) * rows + row) * D + lane * PER;
-            if constexpr (PER % 4 == 0) {
-#pragma unroll
-                for (int e = 0; e < PER; e += 4) {
-                    const float4 v4 = __ldg(reinterpret_cast<const float4*>(src + e));
-                    acc[e] += w * v4.x;
-                    acc[e + 1] += w * v4.y;
-                    acc[e + 2] += w * v4.z;
-                    acc[e + 3] += w * v4.w;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] += w * __ldg(src + e);
-            }
-        }
-    }
-    __nv_bfloat16* dst = out + row * D + lane * PER;
-    if constexpr (PER == 1) {
-        dst[0] = __float2bfloat16_rn(acc[0]);
-    } else {
-#pragma unroll
-        for (int e = 0; e < PER; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
-    }
-    if (lane == 0 && lse != nullptr) lse[row] = L;
+    combine_row<D, false>(part_out, part_lse, C, rows, row, out, lse, threadIdx.x & 31);
 }
 
 }  // namespace attn
@@ -1052,6 +1103,38 @@ attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v, c
     Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
     prm.part_out = part_out;
     prm.part_lse = part_lse;
+    prm.num_splits = num_splits;
+    prm.chunk_len = attn_split_chunk_len(Tk, num_splits);
+    return dispatch_fwd<true>(D, q, k, v, prm, stream);
+}
+
+size_t attn_split_counter_offset(int num_splits, int B, int H, int Tq, int D) {
+    const size_t ws = attn_split_workspace_bytes(num_splits, B, H, Tq, D);
+    return ws == 0 ? 0 : (ws + 255) / 256 * 256;
+}
+
+size_t attn_split_fused_workspace_bytes(int num_splits, int B, int H, int Tq, int D) {
+    const size_t off = attn_split_counter_offset(num_splits, B, H, Tq, D);
+    if (off == 0) return 0;
+    return off + static_cast<size_t>(B) * H * ((static_cast<size_t>(Tq) + BM - 1) / BM) * sizeof(int32_t);
+}
+
+attn_status attn_prefix_fwd_split_fused(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                                        int num_splits, void* workspace, void* out, float* lse, int B, int H,
+                                        int Tq, int Tk, int D, float scale, cudaStream_t stream) {
+    attn_status st = check_args(q, k, v, kv_len, out, B, H, Tq, Tk, D, scale);
+    if (st != ATTN_OK) return st;
+    if (!workspace || !aligned16(workspace) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return ATTN_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_device()) != ATTN_OK) return st;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    prm.part_out = reinterpret_cast<float*>(ws);
+    prm.part_lse = reinterpret_cast<float*>(ws + attn_split_lse_offset(num_splits, B, H, Tq, D));
+    prm.counters = reinterpret_cast<int*>(ws + attn_split_counter_offset(num_splits, B, H, Tq, D));
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
     prm.num_splits = num_splits;
     prm.chunk_len = attn_split_chunk_len(Tk, num_splits);
     return dispatch_fwd<true>(D, q, k, v, prm, stream);

@@ -69,7 +69,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     uint8_t* sQ = smem;
     uint8_t* sKV = smem + C::Q_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::NSLOTS * C::SLOT);
-    uint32_t* words = reinterpret_cast<uint32_t*>(bars + PB_NUM);   // tmem, abort, relay seq
+    uint32_t* words = reinterpret_cast<uint32_t*>(bars + PB_NUM);   // tmem, abort, relay seq, fused-combine flag
     volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
     const uint32_t bar0 = smem_u32(bars);
     const uint32_t sQ_addr = smem_u32(sQ);
@@ -446,6 +446,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+    if constexpr (SPLIT) {
+        if (p.counters != nullptr)
+            fused_combine_tail<D>(p, bh, q0, tid, C::THREADS, reinterpret_cast<volatile int*>(words + 3));
     }
 #undef PBAR
 }

@@ -118,3 +118,21 @@ def test_product_never_imports_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"\b(import|from)\s+oracle\b|attn_oracle|liboracle", text), fn
+
+
+def test_fused_split_geometry_and_argument_checks(lib):
+    C, B, H, Tq, D = 64, 1, 8, 1024, 256
+    ws = lib.attn_split_workspace_bytes(C, B, H, Tq, D)
+    off = lib.attn_split_counter_offset(C, B, H, Tq, D)
+    assert off >= ws and off % 256 == 0 and off - ws < 256
+    # one int32 counter per 128-row query tile of every (b, h)
+    assert lib.attn_split_fused_workspace_bytes(C, B, H, Tq, D) == off + B * H * 8 * 4
+    assert lib.attn_split_fused_workspace_bytes(3, 2, 3, 300, 64) == \
+        lib.attn_split_counter_offset(3, 2, 3, 300, 64) + 2 * 3 * 3 * 4
+    assert lib.attn_split_fused_workspace_bytes(0, 1, 1, 8, 64) == 0
+    f = lib.attn_prefix_fwd_split_fused
+    assert f(A, A, A, A, 4, NULL, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1        # no workspace
+    assert f(A, A, A, A, 4, ctypes.c_void_p(0x10008), A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1  # misaligned
+    assert f(A, A, A, A, 0, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1           # num_splits 0
+    assert f(A, A, A, A, 4, A, NULL, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1        # no out
+    assert f(A, A, A, A, 4, A, A, NULL, 1, 1, 8, 8, 96, 0.1, NULL) == 2           # head dim
