@@ -32,7 +32,7 @@
  *   - Key and value slots at or beyond kv_len[b] are never used: any content there,
  *     NaN and Inf included, leaves out and lse bit-identical.
  *   - kv_len[b] = 0 gives out = 0 and lse = -inf for every row of that element.
- *   - Supported head dims: D in {32, 64, 256}.  Device: compute capability 10.0.
+ *   - Supported head dims: D in {32, 64, 128, 256}.  Device: compute capability 10.0.
  */
 #ifndef ATTN_PREFIX_H
 #define ATTN_PREFIX_H
@@ -48,7 +48,7 @@ extern "C" {
 typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, non-positive size, bad scale */
-    ATTN_ERR_UNSUPPORTED = 2,   /* head dim not in {32,64,256}, or device not sm_100 */
+    ATTN_ERR_UNSUPPORTED = 2,   /* head dim not in {32,64,128,256}, or device not sm_100 */
     ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, attribute) */
     ATTN_ERR_TIMEOUT = 4,       /* a bounded in-kernel wait gave up (device flag) */
     ATTN_ERR_KVLEN_RANGE = 5    /* some kv_len[b] was outside [0, Tk] (device flag) */

@@ -4,7 +4,7 @@
     out, lse = attn_prefix_fwd_splitkv(q, k, v, kv_len, num_splits=64)      # split + combine
     out, lse = attn_prefix_fwd_split_fused(q, k, v, kv_len, num_splits=64)  # one launch
 
-q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 256}; kv_len:
+q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 128, 256}; kv_len:
 int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never take part).
 The computation runs in the hand-written kernels of the C library built from csrc/;
 this package only marshals arguments.

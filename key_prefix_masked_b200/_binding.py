@@ -24,7 +24,7 @@ ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_KVLEN_RANGE = 5
 ATTN_DEBUG_DROP_COPY = 1
 
-SUPPORTED_HEAD_DIMS = (32, 64, 256)
+SUPPORTED_HEAD_DIMS = (32, 64, 128, 256)
 
 # Every symbol the header exports, with its ctypes signature.
 _P = ctypes.c_void_p

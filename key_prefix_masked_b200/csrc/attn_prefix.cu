@@ -939,7 +939,7 @@ attn_status check_args(const void* q, const void* k, const void* v, const void* 
     if (B <= 0 || H <= 0 || Tq <= 0 || Tk <= 0) return ATTN_ERR_INVALID_ARG;
     if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     if (!isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-    if (D != 32 && D != 64 && D != 256) return ATTN_ERR_UNSUPPORTED;
+    if (D != 32 && D != 64 && D != 128 && D != 256) return ATTN_ERR_UNSUPPORTED;
     return ATTN_OK;
 }
 
@@ -1033,6 +1033,7 @@ attn_status dispatch_fwd(int D, const void* q, const void* k, const void* v, con
     switch (D) {
         case 32: return launch_fwd<32, SPLIT>(q, k, v, prm, stream);
         case 64: return launch_fwd<64, SPLIT>(q, k, v, prm, stream);
+        case 128: return launch_fwd<128, SPLIT>(q, k, v, prm, stream);
         case 256:
             if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<256, SPLIT>(q, k, v, prm, stream);
             return launch_fwd_pair<SPLIT>(q, k, v, prm, stream);
@@ -1147,7 +1148,7 @@ attn_status attn_lse_combine(const float* part_out, const float* part_lse, int n
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return ATTN_ERR_INVALID_ARG;
     if (num_splits < 1 || num_splits > 1024 || B <= 0 || H <= 0 || Tq <= 0) return ATTN_ERR_INVALID_ARG;
-    if (D != 32 && D != 64 && D != 256) return ATTN_ERR_UNSUPPORTED;
+    if (D != 32 && D != 64 && D != 128 && D != 256) return ATTN_ERR_UNSUPPORTED;
     attn_status st = check_device();
     if (st != ATTN_OK) return st;
     const long long rows = static_cast<long long>(B) * H * Tq;
@@ -1157,6 +1158,7 @@ attn_status attn_lse_combine(const float* part_out, const float* part_lse, int n
     switch (D) {
         case 32: attn::lse_combine_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
         case 64: attn::lse_combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
+        case 128: attn::lse_combine_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
         default: attn::lse_combine_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;

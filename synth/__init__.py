@@ -58,6 +58,10 @@ WORKLOADS = {
     # a reduced icl shape for profiler captures: same head dim, padding and value
     # distribution, inputs (161 MB) still larger than the L2
     "icl_profile": Workload("icl_profile", 1, 8, 256, 8192, 16512, (16384,), 0.5, True),
+    # head dim 128 (beyond the pages' 64 and 256): the unmasked shape with D=128, and a
+    # prefix-masked one with NaN padding
+    "unmasked_d128": Workload("unmasked_d128", 1, 12, 128, 13622, 13622, (13622,), 1.0, False),
+    "prefix_d128": Workload("prefix_d128", 2, 16, 128, 16384, 16512, (16384, 9001), 1.0, True),
 }
 
 

@@ -61,7 +61,7 @@ def _fwd(lib, q=A, k=A, v=A, kv=A, out=A, lse=NULL, B=1, H=1, Tq=8, Tk=8, D=64, 
     (dict(B=0), 1), (dict(H=-1), 1), (dict(Tq=0), 1), (dict(Tk=0), 1),
     (dict(B=65536, H=65536), 1),                    # B*H overflows int32
     (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
-    (dict(D=128), 2), (dict(D=48), 2), (dict(D=0), 2),
+    (dict(D=96), 2), (dict(D=48), 2), (dict(D=0), 2),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, want):
     assert _fwd(lib, **kw) == want

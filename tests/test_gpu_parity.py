@@ -62,7 +62,7 @@ SWEEP = [
 ]
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("shape", SWEEP, ids=lambda s: "B{}H{}Tq{}Tk{}kv{}".format(
     s[0], s[1], s[2], s[3], "-".join(map(str, s[4]))))
 def test_sweep_against_oracle(kp, D, shape):
@@ -79,7 +79,7 @@ def test_scale_variants(kp, D):
         _run_and_compare(kp, case)
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_padding_content_is_never_read(kp, D):
     lens = (77, 200, 129)
     base = synth.random_case(3, 2, 140, 256, D, lens, seed=3)
@@ -106,7 +106,7 @@ def test_ragged_equals_per_element_calls(kp, D):
         assert bits_equal(o1[0], out[b]) and bits_equal(l1[0], lse[b]), b
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_padded_buffer_equals_truncated_buffer(kp, D):
     for n in (1, 100, 128, 129, 255):
         case = _cuda(synth.random_case(1, 2, 130, 300, D, (n,), seed=n))
@@ -117,7 +117,7 @@ def test_padded_buffer_equals_truncated_buffer(kp, D):
         assert bits_equal(out, o2) and bits_equal(lse, l2), n
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_closed_forms(kp, D):
     case = _cuda(synth.random_case(2, 2, 140, 300, D, (1, 290), seed=9))
     v = torch.full_like(case["v"], 0.3125)
@@ -132,7 +132,7 @@ def test_closed_forms(kp, D):
 
 
 def test_empty_element_exact(kp):
-    for D in (32, 64, 256):
+    for D in (32, 64, 128, 256):
         case = _cuda(synth.random_case(2, 3, 200, 256, D, (0, 256), seed=10))
         out, lse = kp.attn_prefix_fwd(case["q"], case["k"], case["v"], case["kv_len"])
         assert torch.equal(out[0], torch.zeros_like(out[0]))
@@ -151,7 +151,7 @@ def test_kv_len_out_of_range_is_clamped_and_flagged(kp):
     assert torch.equal(out[1], torch.zeros_like(out[1])) and torch.isneginf(lse[1]).all()
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("C", [1, 3, 7])
 def test_split_partials_against_oracle_chunks(kp, D, C):
     lens = (700, 129, 0)
@@ -226,3 +226,11 @@ def test_workload_ragged(kp):
 
 def test_workload_splitkv(kp):
     _workload_check(kp, "splitkv", n_random=0, splits=64)
+
+
+def test_workload_unmasked_d128(kp):
+    _workload_check(kp, "unmasked_d128", n_random=24)
+
+
+def test_workload_prefix_d128(kp):
+    _workload_check(kp, "prefix_d128", n_random=16)

@@ -45,7 +45,7 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("C", [1, 3, 7])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}H{}Tq{}Tk{}".format(*s[:4]))
 def test_fused_equals_two_launch_and_oracle(kp, D, C, shape):
