@@ -8,6 +8,7 @@ from .oracle import (  # noqa: F401
     build_oracle,
     attn_prefix,
     attn_chunk,
+    attn_segments,
     attn_masked,
     lse_combine,
     num_threads,

@@ -266,3 +266,99 @@ int oracle_lse_combine(const double* part_out, const double* part_lse, int C, lo
     }
     return 0;
 }
+
+/* Multi-range key mask: batch element b attends to the keys of its S segments,
+ *   [seg_start[b*S + s], seg_start[b*S + s] + seg_len[b*S + s]),   s = 0 .. S-1,
+ * taken in segment order (the softmax does not depend on the order).  This is the
+ * gathered-shards case of "Add sequence-parallel multi-GPU inference ...", section
+ * "Sequence-parallel inference": each device's context K/V is gathered with padded key
+ * slots, so the valid keys are one range per shard rather than one prefix.
+ * Readings where the pages are silent (listed in the design doc):
+ *   - a segment is intersected with [0, Tk); a negative length counts as 0;
+ *   - a key that lies in two segments takes part twice (the segments are concatenated);
+ *   - the concatenation is cut after Tk keys;
+ *   - no valid key gives out = 0 and lse = -inf, as for an empty prefix.
+ * Keys outside every segment are never read.  out: [B,H,n_rows,D]; lse: [B,H,n_rows]. */
+int oracle_attn_segments(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const int32_t* seg_start, const int32_t* seg_len, int S,
+                         int B, int H, int Tq, int Tk, int D, double scale,
+                         const int64_t* rows, int n_rows, double* out, double* lse) {
+    if (!q || !k || !v || !seg_start || !seg_len || !out || !lse) return -1;
+    if (S <= 0 || B <= 0 || H <= 0 || Tq <= 0 || Tk <= 0 || D <= 0 || n_rows <= 0) return -1;
+    if (!rows && n_rows != Tq) return -1;
+    if (rows)
+        for (int r = 0; r < n_rows; ++r)
+            if (rows[r] < 0 || rows[r] >= Tq) return -1;
+
+    /* the key index list of every batch element */
+    long* keys = (long*)malloc(sizeof(long) * (size_t)B * (size_t)Tk);
+    long* n_keys = (long*)malloc(sizeof(long) * (size_t)B);
+    if (!keys || !n_keys) {
+        free(keys);
+        free(n_keys);
+        return -1;
+    }
+    for (int b = 0; b < B; ++b) {
+        long n = 0;
+        for (int s = 0; s < S && n < Tk; ++s) {
+            long lo = seg_start[(size_t)b * S + s];
+            long len = seg_len[(size_t)b * S + s];
+            long hi = len > 0 ? lo + len : lo;
+            if (lo < 0) lo = 0;
+            if (hi > Tk) hi = Tk;
+            for (long j = lo; j < hi && n < Tk; ++j) keys[(size_t)b * Tk + n++] = j;
+        }
+        n_keys[b] = n;
+    }
+
+    int failed = 0;
+    long total = (long)B * H * n_rows;
+#pragma omp parallel
+    {
+        double* w = (double*)malloc(sizeof(double) * (size_t)Tk);
+        if (!w) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (long idx = 0; idx < total; ++idx) {
+            if (!w) continue;
+            int r = (int)(idx % n_rows);
+            long bh = idx / n_rows;
+            int b = (int)(bh / H);
+            long i = rows ? rows[r] : r;
+            const long* kl = keys + (size_t)b * Tk;
+            long n = n_keys[b];
+            const uint16_t* qrow = q + ((size_t)bh * Tq + (size_t)i) * D;
+            const uint16_t* kbase = k + (size_t)bh * Tk * D;
+            const uint16_t* vbase = v + (size_t)bh * Tk * D;
+            double* o = out + (size_t)idx * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (n == 0) {
+                lse[idx] = -INFINITY;
+                continue;
+            }
+            double m = -INFINITY;
+            for (long t = 0; t < n; ++t) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += widen_bf16(qrow[d]) * widen_bf16(kbase[(size_t)kl[t] * D + d]);
+                w[t] = scale * dot;
+                if (w[t] > m) m = w[t];
+            }
+            double l = 0.0;
+            for (long t = 0; t < n; ++t) {
+                w[t] = exp(w[t] - m);
+                l += w[t];
+            }
+            for (long t = 0; t < n; ++t)
+                for (int d = 0; d < D; ++d) o[d] += w[t] * widen_bf16(vbase[(size_t)kl[t] * D + d]);
+            for (int d = 0; d < D; ++d) o[d] /= l;
+            lse[idx] = m + log(l);
+        }
+        free(w);
+    }
+    free(keys);
+    free(n_keys);
+    return failed ? -1 : 0;
+}

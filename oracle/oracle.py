@@ -58,6 +58,9 @@ def _load():
                                                p, p]
             lib.oracle_attn_masked.restype = i
             lib.oracle_lse_combine.argtypes = [p, p, i, ctypes.c_long, i, p, p]
+            lib.oracle_attn_segments.argtypes = [p, p, p, p, p, i, i, i, i, i, i, ctypes.c_double,
+                                                 p, i, p, p]
+            lib.oracle_attn_segments.restype = i
             lib.oracle_lse_combine.restype = i
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i
@@ -126,6 +129,29 @@ def attn_prefix(q, k, v, kv_len, scale: float, rows=None):
                                 _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_attn_prefix rejected its arguments")
+    return out, lse
+
+
+def attn_segments(q, k, v, seg_start, seg_len, scale: float, rows=None):
+    """Multi-range key mask: batch element b attends to the concatenation of its segments
+    [seg_start[b][s], seg_start[b][s] + seg_len[b][s]) (each cut to [0, Tk), negative
+    lengths as 0, the concatenation cut after Tk keys).  seg_start, seg_len: [B, S] ints.
+    Returns (out float64 [B,H,R,D], lse float64 [B,H,R])."""
+    lib = _load()
+    B, H, Tq, Tk, D = _shape4(q, k)
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    st = np.ascontiguousarray(np.asarray(_to_numpy(seg_start), dtype=np.int32))
+    ln = np.ascontiguousarray(np.asarray(_to_numpy(seg_len), dtype=np.int32))
+    if st.ndim != 2 or st.shape[0] != B or st.shape != ln.shape:
+        raise ValueError("seg_start and seg_len must both be [B, S]")
+    S = int(st.shape[1])
+    r, R = _rows_arg(rows, Tq)
+    out = np.empty((B, H, R, D), dtype=np.float64)
+    lse = np.empty((B, H, R), dtype=np.float64)
+    rc = lib.oracle_attn_segments(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(st), _ptr(ln), S, B, H, Tq, Tk, D,
+                                  float(scale), None if r is None else _ptr(r), R, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_segments rejected its arguments")
     return out, lse
 
 
