@@ -120,6 +120,32 @@ attn_status attn_prefix_fwd_split_fused(const void* q, const void* k, const void
                                         int B, int H, int Tq, int Tk, int D, float scale,
                                         cudaStream_t stream);
 
+/* Multi-range key mask: batch element b attends to the keys of its num_segments (S)
+ * segments instead of one prefix,
+ *     [seg_start[b*S + s], seg_start[b*S + s] + seg_len[b*S + s]),   s = 0 .. S-1,
+ * taken together.  This is the gathered-shards K/V of "Add sequence-parallel multi-GPU
+ * inference ..." (section "Sequence-parallel inference"): every device's context K/V
+ * is gathered with padded key slots, so the valid keys are one range per shard.
+ *   seg_start, seg_len: int32 [B, S], DEVICE memory; the host never reads them.
+ *   S in [1, 4096].  A segment is intersected with [0, Tk); a negative length counts
+ *   as 0; a key in two segments takes part twice; the keys of all segments are cut
+ *   after Tk keys.  A negative length, a non-empty segment reaching outside [0, Tk) or a
+ *   cut raises the sticky ATTN_ERR_KVLEN_RANGE flag.  Slots outside every segment are
+ *   never read: any content there leaves out and lse bit-identical.  An element with no
+ *   valid key gives out = 0, lse = -inf.
+ *   workspace: attn_segments_workspace_bytes(B, H, Tk, D) bytes of device memory,
+ *   16-byte aligned, owned by the caller (no initialisation needed).  One kernel
+ *   gathers the segments' K and V rows into it as a contiguous prefix per element;
+ *   the prefix kernel then runs on the gathered rows (so the result equals
+ *   attn_prefix_fwd on those rows, bit for bit).
+ *   Other arguments and checks as attn_prefix_fwd. */
+size_t attn_segments_workspace_bytes(int B, int H, int Tk, int D);
+attn_status attn_prefix_fwd_segments(const void* q, const void* k, const void* v,
+                                     const int32_t* seg_start, const int32_t* seg_len,
+                                     int num_segments, void* workspace, void* out, float* lse,
+                                     int B, int H, int Tq, int Tk, int D, float scale,
+                                     cudaStream_t stream);
+
 /* Split-KV forward that allocates nothing, for callers that cannot call cudaMalloc.
  * The pages have no counterpart to this entry point: it exists for the integration
  * side, not for the method.  Some callers only ever receive device memory for their

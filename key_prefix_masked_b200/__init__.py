@@ -3,6 +3,7 @@
     out, lse = attn_prefix_fwd(q, k, v, kv_len)          # single pass
     out, lse = attn_prefix_fwd_splitkv(q, k, v, kv_len, num_splits=64)      # split + combine
     out, lse = attn_prefix_fwd_split_fused(q, k, v, kv_len, num_splits=64)  # one launch
+    out, lse = attn_prefix_fwd_segments(q, k, v, seg_start, seg_len)        # multi-range keys
 
 q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 128, 256}; kv_len:
 int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never take part).
@@ -25,6 +26,7 @@ from ._binding import (  # noqa: F401
     fwd_split as attn_prefix_fwd_split,
     fwd_splitkv as attn_prefix_fwd_splitkv,
     fwd_split_fused as attn_prefix_fwd_split_fused,
+    fwd_segments as attn_prefix_fwd_segments,
     fused_workspace,
     lib,
     lse_combine as attn_lse_combine,

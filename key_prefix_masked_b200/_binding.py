@@ -40,6 +40,8 @@ _SIGNATURES = {
     "attn_split_counter_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_split_fused_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_prefix_fwd_split_fused": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "attn_segments_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "attn_prefix_fwd_segments": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_prefix_fwd_splitkv_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
@@ -203,6 +205,44 @@ def fwd_split_fused(q, k, v, kv_len, num_splits, scale=None, workspace=None, out
                                                _ptr(out), _ptr(lse), B, H, Tq, Tk, D, scale,
                                                _stream_ptr(q.device))
     _check(st, "attn_prefix_fwd_split_fused")
+    return out, lse
+
+
+def fwd_segments(q, k, v, seg_start, seg_len, scale=None, workspace=None, out=None, lse=None,
+                 need_lse=True):
+    """Multi-range key mask (attn_prefix_fwd_segments): batch element b attends to the keys
+    of its segments [seg_start[b, s], seg_start[b, s] + seg_len[b, s]).
+
+    seg_start, seg_len: contiguous int32 CUDA tensors [B, S].  `workspace` (uint8, at least
+    attn_segments_workspace_bytes) is allocated here when not given.  Returns (out, lse)."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, T, D]")
+    B = int(q.shape[0])
+    for t, name in ((seg_start, "seg_start"), (seg_len, "seg_len")):
+        if (not t.is_cuda or t.dtype != torch.int32 or t.dim() != 2 or int(t.shape[0]) != B
+                or not t.is_contiguous() or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor [B, S] on q's device")
+    if seg_start.shape != seg_len.shape:
+        raise ValueError("seg_start and seg_len must have the same shape")
+    S = int(seg_start.shape[1])
+    dummy_len = torch.zeros(B, dtype=torch.int32, device=q.device)
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, dummy_len)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    need = int(lib().attn_segments_workspace_bytes(B, H, Tk, D))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if (not workspace.is_cuda or workspace.device != q.device or not workspace.is_contiguous()
+            or workspace.numel() * workspace.element_size() < need):
+        raise ValueError(f"workspace must be a contiguous CUDA buffer of at least {need} bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib().attn_prefix_fwd_segments(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_start), _ptr(seg_len), S,
+                                            _ptr(workspace), _ptr(out), _ptr(lse), B, H, Tq, Tk, D, scale,
+                                            _stream_ptr(q.device))
+    _check(st, "attn_prefix_fwd_segments")
     return out, lse
 
 

@@ -898,6 +898,8 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
     combine_row<D, false>(part_out, part_lse, C, rows, row, out, lse, threadIdx.x & 31);
 }
 
+#include "segments.cuh"
+
 }  // namespace attn
 
 // =========================================================================== host side
@@ -1139,6 +1141,42 @@ attn_status attn_prefix_fwd_split_fused(const void* q, const void* k, const void
     prm.num_splits = num_splits;
     prm.chunk_len = attn_split_chunk_len(Tk, num_splits);
     return dispatch_fwd<true>(D, q, k, v, prm, stream);
+}
+
+size_t attn_segments_workspace_bytes(int B, int H, int Tk, int D) {
+    if (B <= 0 || H <= 0 || Tk <= 0 || D <= 0) return 0;
+    const size_t kv = (static_cast<size_t>(B) * H * Tk * D * 2 + 255) / 256 * 256;
+    return 2 * kv + (static_cast<size_t>(B) * sizeof(int32_t) + 255) / 256 * 256;
+}
+
+attn_status attn_prefix_fwd_segments(const void* q, const void* k, const void* v, const int32_t* seg_start,
+                                     const int32_t* seg_len, int num_segments, void* workspace, void* out,
+                                     float* lse, int B, int H, int Tq, int Tk, int D, float scale,
+                                     cudaStream_t stream) {
+    attn_status st = check_args(q, k, v, seg_start, out, B, H, Tq, Tk, D, scale);
+    if (st != ATTN_OK) return st;
+    if (!seg_len || (reinterpret_cast<uintptr_t>(seg_len) & 3u)) return ATTN_ERR_INVALID_ARG;
+    if (num_segments < 1 || num_segments > attn::SEG_MAX_SEGMENTS) return ATTN_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return ATTN_ERR_INVALID_ARG;
+    const long long n_rb = (static_cast<long long>(Tk) + attn::SEG_ROWS - 1) / attn::SEG_ROWS;
+    const long long grid = n_rb * B * H;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if ((st = check_device()) != ATTN_OK) return st;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const size_t kvb = (static_cast<size_t>(B) * H * Tk * D * 2 + 255) / 256 * 256;
+    uint4* kg = reinterpret_cast<uint4*>(ws);
+    uint4* vg = reinterpret_cast<uint4*>(ws + kvb);
+    int32_t* kvl = reinterpret_cast<int32_t*>(ws + 2 * kvb);
+    const size_t smem = (2 * static_cast<size_t>(num_segments) + 1) * sizeof(int);
+    attn::gather_segments_kernel<<<static_cast<unsigned>(grid), attn::SEG_THREADS, smem, stream>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), kg, vg, seg_start, seg_len, num_segments, H,
+        Tk, D * 2 / 16, static_cast<int>(n_rb), kvl);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    Params prm = base_params(kvl, B, H, Tq, Tk, scale);
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.lse = lse;
+    return dispatch_fwd<false>(D, q, kg, vg, prm, stream);
 }
 
 attn_status attn_lse_combine(const float* part_out, const float* part_lse, int num_splits, void* out, float* lse,

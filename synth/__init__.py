@@ -16,6 +16,10 @@ Workloads (the shapes the pages talk about; no dataset is read):
             N(0,1), padded slots NaN ("Rewrite prefix ...", ragged packed batches)
   splitkv   B=1 H=8 D=256 Tk=1000000 keys, Tq=1024, N(0,0.5^2), 64 key chunks
             ("Add sequence-parallel ...", inducing attention over a huge context)
+  gathered  the icl shape with its 100000 context keys gathered from 4 shards, each
+            padded to 25216 slots (Tk = 100864); valid keys are one range per shard,
+            padded slots NaN ("Add sequence-parallel ...", ICL self-attention over
+            gathered K/V with padded key slots masked)
 """
 from __future__ import annotations
 
@@ -39,6 +43,7 @@ class Workload:
     pad_nan: bool
     num_splits: int = 1
     ragged_seed_draw: bool = False
+    segments: Optional[tuple] = None   # per batch element, ((start, len), ...): multi-range keys
 
     def describe(self) -> dict:
         return {"workload": self.name, "B": self.B, "H": self.H, "D": self.D,
@@ -60,6 +65,8 @@ WORKLOADS = {
     "icl_profile": Workload("icl_profile", 1, 8, 256, 8192, 16512, (16384,), 0.5, True),
     # head dim 128 (beyond the pages' 64 and 256): the unmasked shape with D=128, and a
     # prefix-masked one with NaN padding
+    "gathered": Workload("gathered", 1, 8, 256, 110000, 4 * 25216, (100000,), 0.5, True,
+                         segments=(((0, 25000), (25216, 24800), (50432, 25200), (75648, 25000)),)),
     "unmasked_d128": Workload("unmasked_d128", 1, 12, 128, 13622, 13622, (13622,), 1.0, False),
     "prefix_d128": Workload("prefix_d128", 2, 16, 128, 16384, 16512, (16384, 9001), 1.0, True),
 }
@@ -102,6 +109,44 @@ def fill_padding(k: torch.Tensor, v: torch.Tensor, kv_len: Sequence[int],
             v[b, :, n:, :] = value
 
 
+def segment_mask(segments, B: int, Tk: int) -> torch.Tensor:
+    """[B, Tk] bool: key slot inside one of the batch element's (start, len) ranges."""
+    m = torch.zeros((B, Tk), dtype=torch.bool)
+    for b in range(B):
+        for st, ln in segments[b]:
+            lo, hi = max(int(st), 0), min(int(st) + max(int(ln), 0), Tk)
+            if hi > lo:
+                m[b, lo:hi] = True
+    return m
+
+
+def fill_holes(k: torch.Tensor, v: torch.Tensor, segments, value: float = float("nan")) -> None:
+    """Write `value` into every K/V slot outside the segments (in place)."""
+    holes = ~segment_mask(segments, k.shape[0], k.shape[2]).to(k.device)
+    for b in range(k.shape[0]):
+        k[b][:, holes[b]] = value
+        v[b][:, holes[b]] = value
+
+
+def segment_tensors(segments, device) -> tuple:
+    """seg_start, seg_len as int32 [B, S] tensors on `device`."""
+    st = torch.tensor([[int(a) for a, _ in segs] for segs in segments], dtype=torch.int32, device=device)
+    ln = torch.tensor([[int(n) for _, n in segs] for segs in segments], dtype=torch.int32, device=device)
+    return st, ln
+
+
+def random_segments_case(B: int, H: int, Tq: int, Tk: int, D: int, segments, seed: int = 0,
+                         std: float = 1.0, device="cpu", hole=float("nan")) -> dict:
+    """Seeded q/k/v with key slots outside the segments set to `hole`, plus the
+    segment tensors (int32 [B, S]) and lists."""
+    w = Workload("custom_segments", B, H, D, Tq, Tk, (Tk,) * B, std, False)
+    c = make_inputs(w, device=device, seed=seed)
+    fill_holes(c["k"], c["v"], segments, hole)
+    st, ln = segment_tensors(segments, device)
+    c.update({"seg_start": st, "seg_len": ln, "segments": segments})
+    return c
+
+
 def make_inputs(w: Workload, device="cpu", seed: int = 0, pad_value=None) -> dict:
     """Seeded q, k, v (bf16, [B,H,T,D]) and kv_len (int32 [B]) for a workload.
 
@@ -115,11 +160,19 @@ def make_inputs(w: Workload, device="cpu", seed: int = 0, pad_value=None) -> dic
     k = normal_bf16((w.B, w.H, w.Tk, w.D), w.std, gen, dev)
     v = normal_bf16((w.B, w.H, w.Tk, w.D), w.std, gen, dev)
     pv = pad_value if pad_value is not None else (float("nan") if w.pad_nan else None)
-    if pv is not None:
+    extra = {}
+    if w.segments is not None:
+        # multi-range keys: kv_len is the count of valid keys per element; the holes
+        # between the ranges are the padding
+        if pv is not None:
+            fill_holes(k, v, w.segments, pv)
+        st, ln = segment_tensors(w.segments, dev)
+        extra = {"seg_start": st, "seg_len": ln, "segments": w.segments}
+    elif pv is not None:
         fill_padding(k, v, lens, pv)
     kv = torch.tensor(lens, dtype=torch.int32, device=dev)
     return {"q": q, "k": k, "v": v, "kv_len": kv, "kv_len_list": lens,
-            "scale": default_scale(w.D), "workload": w}
+            "scale": default_scale(w.D), "workload": w, **extra}
 
 
 def random_case(B: int, H: int, Tq: int, Tk: int, D: int, kv_len: Sequence[int],

@@ -136,3 +136,19 @@ def test_fused_split_geometry_and_argument_checks(lib):
     assert f(A, A, A, A, 0, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1           # num_splits 0
     assert f(A, A, A, A, 4, A, NULL, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1        # no out
     assert f(A, A, A, A, 4, A, A, NULL, 1, 1, 8, 8, 96, 0.1, NULL) == 2           # head dim
+
+
+def test_segments_geometry_and_argument_checks(lib):
+    B, H, Tk, D = 2, 3, 1000, 64
+    kv = ((B * H * Tk * D * 2 + 255) // 256) * 256
+    assert lib.attn_segments_workspace_bytes(B, H, Tk, D) == 2 * kv + 256
+    assert lib.attn_segments_workspace_bytes(0, H, Tk, D) == 0
+    f = lib.attn_prefix_fwd_segments
+    #          q  k  v  st len S  ws   out  lse   B  H  Tq Tk  D  scale stream
+    assert f(A, A, A, A, A, 0, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1       # no segments
+    assert f(A, A, A, A, A, 4097, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1    # too many
+    assert f(A, A, A, A, NULL, 2, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1    # no seg_len
+    assert f(A, A, A, NULL, A, 2, A, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1    # no seg_start
+    assert f(A, A, A, A, A, 2, NULL, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1    # no workspace
+    assert f(A, A, A, A, A, 2, ctypes.c_void_p(0x10004), A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1
+    assert f(A, A, A, A, A, 2, A, A, NULL, 1, 1, 8, 8, 96, 0.1, NULL) == 2       # head dim
