@@ -187,6 +187,9 @@ def run_ours(args, rank, world):
     splits = w.num_splits if w.num_splits > 1 else 0
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=dev)
+    segs = w.segments is not None
+    seg_ws = (torch.empty(int(kp.lib().attn_segments_workspace_bytes(w.B, w.H, w.Tk, w.D)), dtype=torch.uint8,
+                          device=dev) if segs else None)
     fused = bool(splits) and args.split_mode == "fused"
     ws = kp.fused_workspace(splits, w.B, w.H, w.Tq, w.D, dev) if fused else None
     parts = ((torch.empty((splits, w.B, w.H, w.Tq, w.D), dtype=torch.float32, device=dev),
@@ -196,7 +199,10 @@ def run_ours(args, rank, world):
     k_ev = []   # separate split mode: events around the split launch (the dominant kernel)
 
     def step(qq, kk, vv, kvl, timed=False):
-        if fused:
+        if segs:
+            kp.attn_prefix_fwd_segments(qq, kk, vv, case["seg_start"], case["seg_len"], scale,
+                                        workspace=seg_ws, out=out, lse=lse)
+        elif fused:
             kp.attn_prefix_fwd_split_fused(qq, kk, vv, kvl, splits, scale, workspace=ws, out=out, lse=lse)
         elif splits:
             if timed:
@@ -210,7 +216,7 @@ def run_ours(args, rank, world):
         else:
             kp.attn_prefix_fwd(qq, kk, vv, kvl, scale, out=out, lse=lse)
 
-    launches_per_step = 2 if (splits and not fused) else 1
+    launches_per_step = 2 if ((splits and not fused) or segs) else 1
     for _ in range(args.warmup):
         step(q, k, v, kv)
     torch.cuda.synchronize()
@@ -245,6 +251,29 @@ def run_ours(args, rank, world):
     step_ms = [a.elapsed_time(b_) for a, b_ in ev]
     total_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
     kern_ms = [a.elapsed_time(b_) for a, b_ in k_ev] if k_ev else step_ms
+    seg_info = None
+    if segs:
+        # the dominant kernel alone: the prefix kernel on the rows the gather left in the
+        # workspace (same launch as inside the step); the rest of the step is the gather
+        kvb = (w.B * w.H * w.Tk * w.D * 2 + 255) // 256 * 256
+        kg = seg_ws[:w.B * w.H * w.Tk * w.D * 2].view(torch.bfloat16).view(w.B, w.H, w.Tk, w.D)
+        vg = seg_ws[kvb:kvb + w.B * w.H * w.Tk * w.D * 2].view(torch.bfloat16).view(w.B, w.H, w.Tk, w.D)
+        kvg = seg_ws[2 * kvb:2 * kvb + 4 * w.B].view(torch.int32)
+        a_ev = []
+        for _ in range(args.steps):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            kp.attn_prefix_fwd(q, kg, vg, kvg, scale, out=out, lse=lse)
+            b_.record(stream)
+            a_ev.append((a, b_))
+        torch.cuda.synchronize()
+        kern_ms = [a.elapsed_time(b_) for a, b_ in a_ev]
+        gather_ms = max(statistics.mean(step_ms) - statistics.mean(kern_ms), 1e-6)
+        gather_bytes = 2 * 2 * sum(case["kv_len_list"]) * w.H * w.D * 2   # K and V rows, read + write
+        seg_info = {"gather_ms": round(gather_ms, 4), "gather_bytes": gather_bytes,
+                    "gather_gbs": round(gather_bytes / gather_ms / 1e6, 1),
+                    "attention_ms": round(statistics.mean(kern_ms), 4),
+                    "note": "gather = step time minus the prefix kernel timed alone on the gathered rows"}
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(flops, world, ms_per_step)
@@ -298,6 +327,7 @@ def run_ours(args, rank, world):
         "step_ms": {"min": round(min(step_ms), 4), "median": round(statistics.median(step_ms), 4),
                     "max": round(max(step_ms), 4)},
         "verified_rows": verified,
+        **({"segments": seg_info} if seg_info else {}),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rec["cpu_baseline"] = cpu_baseline(w, case, args.cpu_seconds)
@@ -312,6 +342,11 @@ def run_e2e(kp, w, case, scale, splits, fused, args, world):
     hk = case["k"].cpu().pin_memory()
     hv = case["v"].cpu().pin_memory()
     hkv = case["kv_len"].cpu().pin_memory()
+    segs = "segments" in case
+    hseg = (case["seg_start"].cpu().pin_memory(), case["seg_len"].cpu().pin_memory()) if segs else ()
+    dseg = tuple(torch.empty_like(case[n]) for n in ("seg_start", "seg_len")) if segs else ()
+    seg_ws = (torch.empty(int(kp.lib().attn_segments_workspace_bytes(w.B, w.H, w.Tk, w.D)), dtype=torch.uint8,
+                          device=dev) if segs else None)
     hout = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
     hlse = torch.empty((w.B, w.H, w.Tq), dtype=torch.float32).pin_memory()
     dq, dk, dv, dkv = (torch.empty_like(case[n]) for n in ("q", "k", "v", "kv_len"))
@@ -328,7 +363,11 @@ def run_e2e(kp, w, case, scale, splits, fused, args, world):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dkv.copy_(hkv, non_blocking=True)
-        if fused:
+        for d_, h_ in zip(dseg, hseg):
+            d_.copy_(h_, non_blocking=True)
+        if segs:
+            kp.attn_prefix_fwd_segments(dq, dk, dv, dseg[0], dseg[1], scale, workspace=seg_ws, out=dout, lse=dlse)
+        elif fused:
             kp.attn_prefix_fwd_split_fused(dq, dk, dv, dkv, splits, scale, workspace=ws, out=dout, lse=dlse)
         elif splits:
             kp.attn_prefix_fwd_split(dq, dk, dv, dkv, splits, scale, *parts)
@@ -351,19 +390,27 @@ def run_e2e(kp, w, case, scale, splits, fused, args, world):
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b_), world) / steps
     flops = workload_flops(w, case["kv_len_list"])
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hkv))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hkv) + tuple(hseg))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
     return {"value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+def _oracle_rows(case, q_rows):
+    """The oracle on some query rows (already selected into q_rows) of a workload case."""
+    import oracle
+    k, v = case["k"].cpu(), case["v"].cpu()
+    if "segments" in case:
+        return oracle.attn_segments(q_rows, k, v, case["seg_start"].cpu(), case["seg_len"].cpu(), case["scale"])
+    return oracle.attn_prefix(q_rows, k, v, case["kv_len_list"], case["scale"])
+
+
 def verify_rows(case, out, lse, w):
     import numpy as np
-    import oracle
     rows = sorted({0, 1, min(127, w.Tq - 1), min(128, w.Tq - 1), w.Tq // 2, w.Tq - 1})
     q = case["q"][:, :, rows].cpu().contiguous()
-    ro, rl = oracle.attn_prefix(q, case["k"].cpu(), case["v"].cpu(), case["kv_len_list"], case["scale"])
+    ro, rl = _oracle_rows(case, q)
     go = out[:, :, rows].float().cpu().double().numpy()
     gl = lse[:, :, rows].cpu().double().numpy()
     ok_out = bool((np.abs(go - ro) <= 1e-2 + 1e-2 * np.abs(ro)).all())
@@ -386,13 +433,11 @@ def traffic_from_profile(workload: str, kernel: str):
 
 # ------------------------------------------------------------------ CPU baseline / reference arm
 def _oracle_sample(w, case, n_rows, seed=0):
-    import oracle
     g = torch.Generator().manual_seed(1234 + seed)
     rows = sorted(set(torch.randint(0, w.Tq, (n_rows,), generator=g).tolist()))
     q = case["q"][:, :, rows].cpu().contiguous()
-    k, v = case["k"].cpu(), case["v"].cpu()
     t = time.perf_counter()
-    oracle.attn_prefix(q, k, v, case["kv_len_list"], case["scale"])
+    _oracle_rows(case, q)
     dt = time.perf_counter() - t
     flops = float(sum(4.0 * w.H * len(rows) * n * w.D for n in case["kv_len_list"]))
     return rows, dt, flops
