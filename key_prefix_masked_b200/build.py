@@ -16,7 +16,7 @@ BUILD_DIR = os.path.join(PKG, "_build")
 LIB_NAME = "libattn_prefix.so"
 LIB_PATH = os.path.join(BUILD_DIR, LIB_NAME)
 SOURCES = ["attn_prefix.cu"]
-HEADERS = ["ptx.cuh", "tmem_ops.cuh", "pair_kernel.cuh", "segments.cuh"]
+HEADERS = ["ptx.cuh", "tmem_ops.cuh", "softmax_math.cuh", "pair_kernel.cuh", "segments.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

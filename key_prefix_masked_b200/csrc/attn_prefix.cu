@@ -46,6 +46,7 @@
 #include "attn_prefix.h"
 #include "ptx.cuh"
 #include "tmem_ops.cuh"
+#include "softmax_math.cuh"
 
 namespace attn {
 
@@ -706,15 +707,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
             }
-            // tree max over the row
-            float mxp[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) mxp[t] = x[t];
-#pragma unroll
-            for (int c = 8; c < BN; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) *
-                             (pos_scale ? sl2 : 1.0f);
+            // row max (three-input maxima)
+            const float mx = row_max(x) * (pos_scale ? sl2 : 1.0f);
             float factor = 1.0f;
             bool rescale = false;
             if (seen == 0) {
@@ -738,17 +732,31 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     if (!ok) break;
                 }
             }
-            float sp[8];
+            // p = 2^(x * mul - m).  One group: the scale-and-shift and the row sum in packed
+            // pairs.  Two-group mode keeps them scalar: its P is held in registers until
+            // the store, and the packed pairs' register alignment then costs spills.
+            float2 sp[4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
+            for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
+            const float2 mul_2 = make_float2(mul, mul);
+            const float2 neg_m2 = make_float2(neg_m, neg_m);
             uint32_t pk[BN / 2];
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
-                    const float p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
-                    sp[e & 7] += p0 + p1;
+                    float p0, p1;
+                    if constexpr (DUAL) {
+                        p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
+                        p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
+                        if (e & 4) sp[e & 3].y += p0 + p1;
+                        else sp[e & 3].x += p0 + p1;
+                    } else {
+                        const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
+                        p0 = fast_exp2(y.x);
+                        p1 = fast_exp2(y.y);
+                        sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
+                    }
                     pk[cc * 16 + e] = pack_bf16x2(p0, p1);
                 }
                 if constexpr (!DUAL) tmem_st16_at(s_addr + cc * 16, &pk[cc * 16]);   // P over S_j
@@ -756,7 +764,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             if constexpr (DUAL) {
                 if (j + 1 < n_tiles) warp_arrive(BAR(BAR_TURN + ((j + 1) & 1)));
             }
-            const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
             l_sum = l_sum * factor + tile_sum;
             // This group's previous PV (PV_{j-2} in two-group mode, else PV_{j-1}) must be
             // complete before O is rescaled, and (two-group mode) before P_w is rewritten.

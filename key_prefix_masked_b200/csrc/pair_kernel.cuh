@@ -326,14 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
             }
-            float mxp[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) mxp[t] = x[t];
-#pragma unroll
-            for (int c = 8; c < BN; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) *
-                             (pos_scale ? sl2 : 1.0f);
+            const float mx = row_max(x) * (pos_scale ? sl2 : 1.0f);   // three-input maxima
             float factor = 1.0f;
             bool rescale = false;
             if (j == 0) {
@@ -346,22 +339,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             }
             const float mul = pos_scale ? sl2 : 1.0f;
             const float neg_m = -m_ref;
-            float sp[8];
+            // p = 2^(x * mul - m): the scale-and-shift and the row sum in packed pairs
+            float2 sp[4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) sp[t] = 0.0f;
+            for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
+            const float2 mul_2 = make_float2(mul, mul);
+            const float2 neg_m2 = make_float2(neg_m, neg_m);
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
-                    const float p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
-                    sp[e & 7] += p0 + p1;
+                    const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
+                    const float p0 = fast_exp2(y.x);
+                    const float p1 = fast_exp2(y.y);
+                    sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(s_addr + cc * 16, pk);
             }
-            const float tile_sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
             l_sum = l_sum * factor + tile_sum;
             if (rescale) {
                 // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last tile
