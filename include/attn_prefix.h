@@ -54,6 +54,18 @@ typedef enum {
     ATTN_ERR_KVLEN_RANGE = 5    /* some kv_len[b] was outside [0, Tk] (device flag) */
 } attn_status;
 
+/* Element strides of a [B, H, T, D] operand whose d index is contiguous (stride 1):
+ * element (b, h, t, d) is at base + b*b_stride + h*h_stride + t*t_stride + d.  The
+ * *_strided entry points take one per operand; NULL means the contiguous [B,H,T,D]
+ * layout (b = H*T*D, h = T*D, t = D).  JAX's [B, T, H, D] ("BTNH") layout is
+ * {T*H*D, D, H*D}; q, k, v sliced out of one packed [B, T, 3, H, D] tensor are
+ * {3*T*H*D, D, 3*H*D}.  Every stride must be a non-negative multiple of 8 elements
+ * (16-byte rows, as TMA and the vector stores need) and t >= D; otherwise the call
+ * returns ATTN_ERR_INVALID_ARG.  Output rows of distinct (b, h, t) must not overlap. */
+typedef struct {
+    int64_t b, h, t;
+} attn_strides;
+
 /* Single-pass forward.
  *   q:      bf16 [B, H, Tq, D]         k, v: bf16 [B, H, Tk, D]
  *   kv_len: int32 [B], device memory  (valid key count per batch element)
@@ -65,6 +77,16 @@ attn_status attn_prefix_fwd(const void* q, const void* k, const void* v,
                             const int32_t* kv_len, void* out, float* lse,
                             int B, int H, int Tq, int Tk, int D, float scale,
                             cudaStream_t stream);
+
+/* attn_prefix_fwd with q, k, v and out at caller strides (see attn_strides); lse stays
+ * contiguous [B, H, Tq].  Same result, bit for bit, as attn_prefix_fwd on contiguous
+ * copies. */
+attn_status attn_prefix_fwd_strided(const void* q, const void* k, const void* v,
+                                    const int32_t* kv_len, void* out, float* lse,
+                                    int B, int H, int Tq, int Tk, int D, float scale,
+                                    const attn_strides* q_strides, const attn_strides* k_strides,
+                                    const attn_strides* v_strides, const attn_strides* out_strides,
+                                    cudaStream_t stream);
 
 /* Keys per split chunk for a given key buffer length and split count: ceil(Tk/C)
  * rounded up to the 128-key tile.  Chunk c covers keys [c*L, min((c+1)*L, kv_len[b])).
@@ -87,6 +109,15 @@ attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v,
                                   int B, int H, int Tq, int Tk, int D, float scale,
                                   cudaStream_t stream);
 
+/* attn_prefix_fwd_split with q, k, v at caller strides; the partials keep the layout
+ * above. */
+attn_status attn_prefix_fwd_split_strided(const void* q, const void* k, const void* v,
+                                          const int32_t* kv_len, int num_splits,
+                                          float* part_out, float* part_lse,
+                                          int B, int H, int Tq, int Tk, int D, float scale,
+                                          const attn_strides* q_strides, const attn_strides* k_strides,
+                                          const attn_strides* v_strides, cudaStream_t stream);
+
 /* Exact log-sum-exp combination of split partials (same layouts as above):
  *   M = max_c lse_c;  lse = M + ln sum_c exp(lse_c - M);  out = sum_c exp(lse_c - lse) O_c
  * Rows whose every partial is empty give out = 0, lse = -inf.
@@ -94,6 +125,10 @@ attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v,
 attn_status attn_lse_combine(const float* part_out, const float* part_lse, int num_splits,
                              void* out, float* lse, int B, int H, int Tq, int D,
                              cudaStream_t stream);
+/* attn_lse_combine writing out at caller strides (lse stays contiguous). */
+attn_status attn_lse_combine_strided(const float* part_out, const float* part_lse, int num_splits,
+                                     void* out, float* lse, int B, int H, int Tq, int D,
+                                     const attn_strides* out_strides, cudaStream_t stream);
 
 /* Split-KV forward with the combine fused into the same launch: the split partials of
  * attn_prefix_fwd_split, then, inside the kernel, the exact combination of

@@ -32,6 +32,9 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 _SIGNATURES = {
     "attn_prefix_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "attn_prefix_fwd_strided": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P]),
+    "attn_prefix_fwd_split_strided": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
+    "attn_lse_combine_strided": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
     "attn_split_chunk_len": (_I, [_I, _I]),
     "attn_split_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "attn_split_lse_offset": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
@@ -95,10 +98,30 @@ def _ptr(t):
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
 
-def _check_qkv(q, k, v, kv_len):
+class _Strides(ctypes.Structure):
+    """attn_strides: element strides along b, h, t of a [B,H,T,D] operand (d contiguous)."""
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("t", ctypes.c_int64)]
+
+
+def _strides_of(t):
+    """The attn_strides of a [B,H,T,D] view whose last dim is contiguous."""
+    sb, sh, st, sd = t.stride()
+    if sd != 1:
+        raise ValueError("the head dim must be contiguous (stride 1)")
+    return _Strides(sb, sh, st)
+
+
+def _strided_ok(t):
+    return t.dim() == 4 and t.stride(3) == 1 and all(x % 8 == 0 for x in t.stride()[:3])
+
+
+def _check_qkv(q, k, v, kv_len, strided=False):
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B,H,T,D]")
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor [B,H,T,D]")
+        if not (t.is_contiguous() or (strided and _strided_ok(t))):
+            raise ValueError(f"{name} must be contiguous, or a [B,H,T,D] view with a contiguous head dim "
+                             "and strides that are multiples of 8 elements")
     B, H, Tq, D = q.shape
     if k.shape[:2] != (B, H) or k.shape[3] != D or v.shape != k.shape:
         raise ValueError("k and v must be [B,H,Tk,D] matching q's B, H, D")
@@ -111,16 +134,29 @@ def _check_qkv(q, k, v, kv_len):
 
 
 def fwd(q, k, v, kv_len, scale=None, out=None, lse=None, need_lse=True):
-    """Prefix-masked attention forward (attn_prefix_fwd): returns (out bf16, lse fp32)."""
-    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len)
+    """Prefix-masked attention forward (attn_prefix_fwd): returns (out bf16, lse fp32).
+
+    q, k, v (and out, if given) may be [B,H,T,D] views of other layouts, e.g.
+    x.transpose(1, 2) of a [B,T,H,D] tensor: their strides go to attn_prefix_fwd_strided.
+    A new out takes q's layout."""
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len, strided=True)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
+    elif (out.shape != q.shape or out.dtype != torch.bfloat16 or out.device != q.device
+          or not (out.is_contiguous() or _strided_ok(out))):
+        raise ValueError("out must be a bf16 [B,H,Tq,D] tensor on q's device with a contiguous head dim")
     if lse is None and need_lse:
         lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
-        st = lib().attn_prefix_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), _ptr(out), _ptr(lse),
-                                   B, H, Tq, Tk, D, scale, _stream_ptr(q.device))
+        if all(t.is_contiguous() for t in (q, k, v, out)):
+            st = lib().attn_prefix_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), _ptr(out), _ptr(lse),
+                                       B, H, Tq, Tk, D, scale, _stream_ptr(q.device))
+        else:
+            s4 = [_strides_of(t) for t in (q, k, v, out)]
+            st = lib().attn_prefix_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), _ptr(out), _ptr(lse),
+                                               B, H, Tq, Tk, D, scale, *[ctypes.addressof(x) for x in s4],
+                                               _stream_ptr(q.device))
     _check(st, "attn_prefix_fwd")
     return out, lse
 
@@ -131,7 +167,7 @@ def split_chunk_len(Tk: int, num_splits: int) -> int:
 
 def fwd_split(q, k, v, kv_len, num_splits, scale=None, part_out=None, part_lse=None):
     """Split-KV partials (attn_prefix_fwd_split): fp32 part_out [C,B,H,Tq,D], part_lse [C,B,H,Tq]."""
-    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len)
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, kv_len, strided=True)
     C = int(num_splits)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if part_out is None:
@@ -139,9 +175,15 @@ def fwd_split(q, k, v, kv_len, num_splits, scale=None, part_out=None, part_lse=N
     if part_lse is None:
         part_lse = torch.empty((C, B, H, Tq), dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
-        st = lib().attn_prefix_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), C, _ptr(part_out),
-                                         _ptr(part_lse), B, H, Tq, Tk, D, scale,
-                                         _stream_ptr(q.device))
+        if all(t.is_contiguous() for t in (q, k, v)):
+            st = lib().attn_prefix_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), C, _ptr(part_out),
+                                             _ptr(part_lse), B, H, Tq, Tk, D, scale,
+                                             _stream_ptr(q.device))
+        else:
+            s3 = [_strides_of(t) for t in (q, k, v)]
+            st = lib().attn_prefix_fwd_split_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_len), C, _ptr(part_out),
+                                                     _ptr(part_lse), B, H, Tq, Tk, D, scale,
+                                                     *[ctypes.addressof(x) for x in s3], _stream_ptr(q.device))
     _check(st, "attn_prefix_fwd_split")
     return part_out, part_lse
 
@@ -157,11 +199,19 @@ def lse_combine(part_out, part_lse, out=None, lse=None, need_lse=True):
         raise ValueError("part_lse must be [C,B,H,Tq]")
     if out is None:
         out = torch.empty((B, H, Tq, D), dtype=torch.bfloat16, device=part_out.device)
+    elif (tuple(out.shape) != (B, H, Tq, D) or out.dtype != torch.bfloat16 or out.device != part_out.device
+          or not (out.is_contiguous() or _strided_ok(out))):
+        raise ValueError("out must be a bf16 [B,H,Tq,D] tensor with a contiguous head dim")
     if lse is None and need_lse:
         lse = torch.empty((B, H, Tq), dtype=torch.float32, device=part_out.device)
     with torch.cuda.device(part_out.device):
-        st = lib().attn_lse_combine(_ptr(part_out), _ptr(part_lse), C, _ptr(out), _ptr(lse),
-                                    B, H, Tq, D, _stream_ptr(part_out.device))
+        if out.is_contiguous():
+            st = lib().attn_lse_combine(_ptr(part_out), _ptr(part_lse), C, _ptr(out), _ptr(lse),
+                                        B, H, Tq, D, _stream_ptr(part_out.device))
+        else:
+            so = _strides_of(out)
+            st = lib().attn_lse_combine_strided(_ptr(part_out), _ptr(part_lse), C, _ptr(out), _ptr(lse),
+                                                B, H, Tq, D, ctypes.addressof(so), _stream_ptr(part_out.device))
     _check(st, "attn_lse_combine")
     return out, lse
 

@@ -116,11 +116,12 @@ enum : int {
 
 struct Params {
     const int32_t* kv_len;
-    __nv_bfloat16* out;   // single pass, or split with fused combine: bf16 [B,H,Tq,D]
+    __nv_bfloat16* out;   // single pass, or split with fused combine: bf16 [B,H,Tq,D] at strides out_s*
     float* lse;           // single pass, or split with fused combine: fp32 [B,H,Tq] or null
     float* part_out;      // split: fp32 [C,B,H,Tq,D]
     float* part_lse;      // split: fp32 [C,B,H,Tq]
     int* counters;        // split with fused combine: int32 [B*H*ceil(Tq/128)], else null
+    long long out_sb, out_sh, out_st;   // element strides of out along b, h, t (d contiguous)
     int B, H, Tq, Tk;
     int n_qtiles;
     int num_splits;
@@ -202,7 +203,8 @@ __device__ __noinline__ bool wait_bar_drain_cl(uint32_t bar, uint32_t parity, un
 // Exact combination of one row's split partials, by one warp (lane = thread % 32):
 //   M = max_c lse_c,  lse = M + ln sum_c exp(lse_c - M),  out = sum_c exp(lse_c - lse) O_c,
 // the log-sum-exp rule of split-KV; a row whose every chunk is empty gives 0 / -inf.
-// Partials are [C][rows][D] and [C][rows].  FRESH: the partials were written by other
+// Partials are [C][rows][D] and [C][rows]; out_row points at the row's D outputs, lse
+// is indexed by row.  FRESH: the partials were written by other
 // CTAs of the running kernel, so they are read through L2 (ld.global.cg) instead of the
 // read-only path; the arithmetic, and so the result, is the same either way.
 template <typename T, bool FRESH>
@@ -212,7 +214,7 @@ __device__ __forceinline__ T ld_part(const T* ptr) {
 }
 template <int D, bool FRESH>
 __device__ __forceinline__ void combine_row(const float* __restrict__ part_out, const float* __restrict__ part_lse,
-                                            int C, long long rows, long long row, __nv_bfloat16* __restrict__ out,
+                                            int C, long long rows, long long row, __nv_bfloat16* __restrict__ out_row,
                                             float* __restrict__ lse, int lane) {
     constexpr int PER = D / 32;
     float M = -INFINITY;
@@ -248,7 +250,7 @@ __device__ __forceinline__ void combine_row(const float* __restrict__ part_out, 
             }
         }
     }
-    __nv_bfloat16* dst = out + row * D + lane * PER;
+    __nv_bfloat16* dst = out_row + lane * PER;
     if constexpr (PER == 1) {
         dst[0] = __float2bfloat16_rn(acc[0]);
     } else {
@@ -282,9 +284,10 @@ __device__ __forceinline__ void fused_combine_tail(const Params& p, int bh, int 
     __threadfence();          // the other chunks' partials, counted in before the count completed
     const long long rows = static_cast<long long>(p.B) * p.H * p.Tq;
     const int nr = min(BM, p.Tq - q0);
+    const int b = bh / p.H, h = bh - b * p.H;
     for (int r = t >> 5; r < nr; r += nthreads >> 5)
         combine_row<D, true>(p.part_out, p.part_lse, p.num_splits, rows, static_cast<long long>(bh) * p.Tq + q0 + r,
-                             p.out, p.lse, t & 31);
+                             p.out + b * p.out_sb + h * p.out_sh + (q0 + r) * p.out_st, p.lse, t & 31);
 }
 
 template <int D, bool SPLIT>
@@ -318,6 +321,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     const int split = SPLIT ? unit % p.num_splits : 0;
     const int bh = SPLIT ? unit / p.num_splits : unit;
     const int b = bh / p.H;
+    const int h = bh - b * p.H;
     const int q0 = qtile * BM;
 
     int kv = __ldg(p.kv_len + b);
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             mbar_arrive_expect_tx(BAR(BAR_Q), C::Q_BYTES);
 #pragma unroll
             for (int blk = 0; blk < C::NBLK; ++blk)
-                tma_load_3d(sQ_addr + blk * BM * C::SW, &tm_q, blk * C::BLK, q0, bh, BAR(BAR_Q));
+                tma_load_4d(sQ_addr + blk * BM * C::SW, &tm_q, blk * C::BLK, q0, h, b, BAR(BAR_Q));
 
             int gi = 0;
             uint32_t phase = 0;
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                             dropped = gi;   // announced, never issued: the consumer's wait runs out
                             continue;
                         }
-                        tma_load_3d(sKV_addr + (gi * C::GRP + cc) * C::SLOT, &tm_k, c * C::BLK, key0, bh,
+                        tma_load_4d(sKV_addr + (gi * C::GRP + cc) * C::SLOT, &tm_k, c * C::BLK, key0, h, b,
                                     BAR(BAR_FULL + gi));
                     }
                     release_slot_bookkeeping();
@@ -424,8 +428,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         const int c = g * C::GRP + cc;
 #pragma unroll
                         for (int blk = 0; blk < C::NBLK; ++blk)
-                            tma_load_3d(sKV_addr + (gi * C::GRP + cc) * C::SLOT + blk * C::V_ROWS * C::SW, &tm_v,
-                                        blk * C::BLK, key0 + c * C::V_ROWS, bh, BAR(BAR_FULL + gi));
+                            tma_load_4d(sKV_addr + (gi * C::GRP + cc) * C::SLOT + blk * C::V_ROWS * C::SW, &tm_v,
+                                        blk * C::BLK, key0 + c * C::V_ROWS, h, b, BAR(BAR_FULL + gi));
                     }
                     release_slot_bookkeeping();
                 }
@@ -859,7 +863,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     *reinterpret_cast<float4*>(dst + e) = v4;
                 }
             } else {
-                __nv_bfloat16* dst = p.out + (static_cast<long long>(bh) * p.Tq + row) * D + oc * 32;
+                __nv_bfloat16* dst = p.out + b * p.out_sb + h * p.out_sh + row * p.out_st + oc * 32;
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint4 v4;
@@ -895,15 +899,18 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 
 #include "pair_kernel.cuh"
 
-// One warp per output row (see combine_row).
+// One warp per output row (see combine_row); out at element strides (sb, sh, st).
 template <int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_out,
                                                           const float* __restrict__ part_lse, int C,
-                                                          long long rows, __nv_bfloat16* __restrict__ out,
-                                                          float* __restrict__ lse) {
+                                                          long long rows, int H, int Tq,
+                                                          __nv_bfloat16* __restrict__ out, long long sb,
+                                                          long long sh, long long st, float* __restrict__ lse) {
     const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (row >= rows) return;
-    combine_row<D, false>(part_out, part_lse, C, rows, row, out, lse, threadIdx.x & 31);
+    const long long bh = row / Tq, q = row - bh * Tq;
+    const long long b = bh / H, h = bh - b * H;
+    combine_row<D, false>(part_out, part_lse, C, rows, row, out + b * sb + h * sh + q * st, lse, threadIdx.x & 31);
 }
 
 #include "segments.cuh"
@@ -939,6 +946,26 @@ EncodeTiledFn encode_fn() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Element strides of one [B, H, T, D] operand (d contiguous).
+struct Strides {
+    long long b, h, t;
+};
+Strides contiguous(int H, int T, int D) {
+    return {static_cast<long long>(H) * T * D, static_cast<long long>(T) * D, static_cast<long long>(D)};
+}
+// Caller strides, or the contiguous [B,H,T,D] layout for NULL.  Every stride must be a
+// non-negative multiple of 8 elements (16-byte rows for TMA and vector stores), and a
+// row may not overlap the next one (t >= D).
+bool resolve_strides(const attn_strides* in, int H, int T, int D, Strides* out) {
+    if (in == nullptr) {
+        *out = contiguous(H, T, D);
+        return true;
+    }
+    if (in->b < 0 || in->h < 0 || in->t < D || (in->b & 7) || (in->h & 7) || (in->t & 7)) return false;
+    *out = {static_cast<long long>(in->b), static_cast<long long>(in->h), static_cast<long long>(in->t)};
+    return true;
+}
 
 // Host checks that need no CUDA call.
 attn_status check_args(const void* q, const void* k, const void* v, const void* kv_len, const void* out,
@@ -979,28 +1006,34 @@ attn_status check_device() {
 }
 
 // 3-D map over a [B*H, T, D] bf16 tensor; box = (swizzle block columns, rows, 1).
-bool make_map(CUtensorMap* map, const void* base, int T, long long BH, int D, int box_cols, int box_rows,
-              CUtensorMapSwizzle swz) {
+// A [B, H, T, D] bf16 tensor at element strides s (d contiguous) as a 4-D TMA map with
+// dims (D, T, H, B); a box is box_rows rows x box_cols columns of one (b, h).
+bool make_map(CUtensorMap* map, const void* base, int B, int H, int T, int D, const Strides& s, int box_cols,
+              int box_rows, CUtensorMapSwizzle swz) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2ull, static_cast<cuuint64_t>(T) * D * 2ull};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.t) * 2ull, static_cast<cuuint64_t>(s.h) * 2ull,
+                             static_cast<cuuint64_t>(s.b) * 2ull};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 template <int D, bool SPLIT>
-attn_status launch_fwd(const void* q, const void* k, const void* v, Params prm, cudaStream_t stream) {
+attn_status launch_fwd(const void* q, const void* k, const void* v, const Strides* st, Params prm,
+                       cudaStream_t stream) {
     using C = Cfg<D>;
     const long long BH = static_cast<long long>(prm.B) * prm.H;
     const CUtensorMapSwizzle swz = (C::SW == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, prm.Tq, BH, D, C::BLK, BM, swz) || !make_map(&mk, k, prm.Tk, BH, D, C::BLK, BN, swz) ||
-        !make_map(&mv, v, prm.Tk, BH, D, C::BLK, C::V_ROWS, swz))
+    if (!make_map(&mq, q, prm.B, prm.H, prm.Tq, D, st[0], C::BLK, BM, swz) ||
+        !make_map(&mk, k, prm.B, prm.H, prm.Tk, D, st[1], C::BLK, BN, swz) ||
+        !make_map(&mv, v, prm.B, prm.H, prm.Tk, D, st[2], C::BLK, C::V_ROWS, swz))
         return ATTN_ERR_CUDA;
     const long long grid = static_cast<long long>(prm.n_qtiles) * BH * (SPLIT ? prm.num_splits : 1);
     if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
@@ -1016,13 +1049,14 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, Params prm, 
 
 // Head dim 256 runs on CTA pairs: 256-row query tiles, each CTA copying half of K and V.
 template <bool SPLIT>
-attn_status launch_fwd_pair(const void* q, const void* k, const void* v, Params prm, cudaStream_t stream) {
+attn_status launch_fwd_pair(const void* q, const void* k, const void* v, const Strides* st, Params prm,
+                            cudaStream_t stream) {
     using C = attn::PairCfg;
     const long long BH = static_cast<long long>(prm.B) * prm.H;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, prm.Tq, BH, C::D, 64, C::ROWS, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, k, prm.Tk, BH, C::D, 64, C::KH, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, v, prm.Tk, BH, C::D, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map(&mq, q, prm.B, prm.H, prm.Tq, C::D, st[0], 64, C::ROWS, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, k, prm.B, prm.H, prm.Tk, C::D, st[1], 64, C::KH, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, v, prm.B, prm.H, prm.Tk, C::D, st[2], 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return ATTN_ERR_CUDA;
     prm.n_qtiles = (prm.Tq + 2 * C::ROWS - 1) / (2 * C::ROWS);
     const long long grid = 2LL * prm.n_qtiles * BH * (SPLIT ? prm.num_splits : 1);
@@ -1037,21 +1071,24 @@ attn_status launch_fwd_pair(const void* q, const void* k, const void* v, Params 
     return ATTN_OK;
 }
 
+// st: strides of q, k, v (NULL: all contiguous).
 template <bool SPLIT>
 attn_status dispatch_fwd(int D, const void* q, const void* k, const void* v, const Params& prm,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const Strides* st = nullptr) {
+    Strides dflt[3] = {contiguous(prm.H, prm.Tq, D), contiguous(prm.H, prm.Tk, D), contiguous(prm.H, prm.Tk, D)};
+    if (st == nullptr) st = dflt;
     switch (D) {
-        case 32: return launch_fwd<32, SPLIT>(q, k, v, prm, stream);
-        case 64: return launch_fwd<64, SPLIT>(q, k, v, prm, stream);
-        case 128: return launch_fwd<128, SPLIT>(q, k, v, prm, stream);
+        case 32: return launch_fwd<32, SPLIT>(q, k, v, st, prm, stream);
+        case 64: return launch_fwd<64, SPLIT>(q, k, v, st, prm, stream);
+        case 128: return launch_fwd<128, SPLIT>(q, k, v, st, prm, stream);
         case 256:
-            if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<256, SPLIT>(q, k, v, prm, stream);
-            return launch_fwd_pair<SPLIT>(q, k, v, prm, stream);
+            if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<256, SPLIT>(q, k, v, st, prm, stream);
+            return launch_fwd_pair<SPLIT>(q, k, v, st, prm, stream);
         default: return ATTN_ERR_UNSUPPORTED;
     }
 }
 
-Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, float scale) {
+Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, int D, float scale) {
     Params prm;
     memset(&prm, 0, sizeof prm);
     prm.kv_len = kv_len;
@@ -1063,6 +1100,10 @@ Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, float sc
     prm.num_splits = 1;
     prm.chunk_len = Tk;
     prm.scale_log2 = scale * attn::LOG2E;
+    const Strides so = contiguous(H, Tq, D);   // out: contiguous [B,H,Tq,D] unless set otherwise
+    prm.out_sb = so.b;
+    prm.out_sh = so.h;
+    prm.out_st = so.t;
     prm.wait_ns = g_wait_ns;
     prm.debug = g_debug;
     return prm;
@@ -1072,16 +1113,32 @@ Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, float sc
 
 extern "C" {
 
-attn_status attn_prefix_fwd(const void* q, const void* k, const void* v, const int32_t* kv_len, void* out,
-                            float* lse, int B, int H, int Tq, int Tk, int D, float scale, cudaStream_t stream) {
+attn_status attn_prefix_fwd_strided(const void* q, const void* k, const void* v, const int32_t* kv_len, void* out,
+                                    float* lse, int B, int H, int Tq, int Tk, int D, float scale,
+                                    const attn_strides* q_strides, const attn_strides* k_strides,
+                                    const attn_strides* v_strides, const attn_strides* out_strides,
+                                    cudaStream_t stream) {
     attn_status st = check_args(q, k, v, kv_len, out, B, H, Tq, Tk, D, scale);
     if (st != ATTN_OK) return st;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+    Strides s3[3], so;
+    if (!resolve_strides(q_strides, H, Tq, D, &s3[0]) || !resolve_strides(k_strides, H, Tk, D, &s3[1]) ||
+        !resolve_strides(v_strides, H, Tk, D, &s3[2]) || !resolve_strides(out_strides, H, Tq, D, &so))
+        return ATTN_ERR_INVALID_ARG;
     if ((st = check_device()) != ATTN_OK) return st;
-    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    Params prm = base_params(kv_len, B, H, Tq, Tk, D, scale);
     prm.out = static_cast<__nv_bfloat16*>(out);
     prm.lse = lse;
-    return dispatch_fwd<false>(D, q, k, v, prm, stream);
+    prm.out_sb = so.b;
+    prm.out_sh = so.h;
+    prm.out_st = so.t;
+    return dispatch_fwd<false>(D, q, k, v, prm, stream, s3);
+}
+
+attn_status attn_prefix_fwd(const void* q, const void* k, const void* v, const int32_t* kv_len, void* out,
+                            float* lse, int B, int H, int Tq, int Tk, int D, float scale, cudaStream_t stream) {
+    return attn_prefix_fwd_strided(q, k, v, kv_len, out, lse, B, H, Tq, Tk, D, scale, nullptr, nullptr, nullptr,
+                                   nullptr, stream);
 }
 
 int attn_split_chunk_len(int Tk, int num_splits) {
@@ -1103,20 +1160,33 @@ size_t attn_split_workspace_bytes(int num_splits, int B, int H, int Tq, int D) {
     return off + static_cast<size_t>(num_splits) * B * H * Tq * sizeof(float);
 }
 
-attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v, const int32_t* kv_len,
-                                  int num_splits, float* part_out, float* part_lse, int B, int H, int Tq, int Tk,
-                                  int D, float scale, cudaStream_t stream) {
+attn_status attn_prefix_fwd_split_strided(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                                          int num_splits, float* part_out, float* part_lse, int B, int H, int Tq,
+                                          int Tk, int D, float scale, const attn_strides* q_strides,
+                                          const attn_strides* k_strides, const attn_strides* v_strides,
+                                          cudaStream_t stream) {
     attn_status st = check_args(q, k, v, kv_len, part_out, B, H, Tq, Tk, D, scale);
     if (st != ATTN_OK) return st;
     if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u)) return ATTN_ERR_INVALID_ARG;
     if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
+    Strides s3[3];
+    if (!resolve_strides(q_strides, H, Tq, D, &s3[0]) || !resolve_strides(k_strides, H, Tk, D, &s3[1]) ||
+        !resolve_strides(v_strides, H, Tk, D, &s3[2]))
+        return ATTN_ERR_INVALID_ARG;
     if ((st = check_device()) != ATTN_OK) return st;
-    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    Params prm = base_params(kv_len, B, H, Tq, Tk, D, scale);
     prm.part_out = part_out;
     prm.part_lse = part_lse;
     prm.num_splits = num_splits;
     prm.chunk_len = attn_split_chunk_len(Tk, num_splits);
-    return dispatch_fwd<true>(D, q, k, v, prm, stream);
+    return dispatch_fwd<true>(D, q, k, v, prm, stream, s3);
+}
+
+attn_status attn_prefix_fwd_split(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                                  int num_splits, float* part_out, float* part_lse, int B, int H, int Tq, int Tk,
+                                  int D, float scale, cudaStream_t stream) {
+    return attn_prefix_fwd_split_strided(q, k, v, kv_len, num_splits, part_out, part_lse, B, H, Tq, Tk, D, scale,
+                                         nullptr, nullptr, nullptr, stream);
 }
 
 size_t attn_split_counter_offset(int num_splits, int B, int H, int Tq, int D) {
@@ -1140,7 +1210,7 @@ attn_status attn_prefix_fwd_split_fused(const void* q, const void* k, const void
     if (num_splits < 1 || num_splits > 1024) return ATTN_ERR_INVALID_ARG;
     if ((st = check_device()) != ATTN_OK) return st;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    Params prm = base_params(kv_len, B, H, Tq, Tk, scale);
+    Params prm = base_params(kv_len, B, H, Tq, Tk, D, scale);
     prm.part_out = reinterpret_cast<float*>(ws);
     prm.part_lse = reinterpret_cast<float*>(ws + attn_split_lse_offset(num_splits, B, H, Tq, D));
     prm.counters = reinterpret_cast<int*>(ws + attn_split_counter_offset(num_splits, B, H, Tq, D));
@@ -1181,15 +1251,18 @@ attn_status attn_prefix_fwd_segments(const void* q, const void* k, const void* v
         static_cast<const uint4*>(k), static_cast<const uint4*>(v), kg, vg, seg_start, seg_len, num_segments, H,
         Tk, D * 2 / 16, static_cast<int>(n_rb), kvl);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    Params prm = base_params(kvl, B, H, Tq, Tk, scale);
+    Params prm = base_params(kvl, B, H, Tq, Tk, D, scale);
     prm.out = static_cast<__nv_bfloat16*>(out);
     prm.lse = lse;
     return dispatch_fwd<false>(D, q, kg, vg, prm, stream);
 }
 
-attn_status attn_lse_combine(const float* part_out, const float* part_lse, int num_splits, void* out, float* lse,
-                             int B, int H, int Tq, int D, cudaStream_t stream) {
+attn_status attn_lse_combine_strided(const float* part_out, const float* part_lse, int num_splits, void* out,
+                                     float* lse, int B, int H, int Tq, int D, const attn_strides* out_strides,
+                                     cudaStream_t stream) {
     if (!part_out || !part_lse || !out) return ATTN_ERR_INVALID_ARG;
+    Strides so;
+    if (D <= 0 || !resolve_strides(out_strides, H, Tq, D, &so)) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(part_out) || !aligned16(out) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return ATTN_ERR_INVALID_ARG;
@@ -1201,14 +1274,20 @@ attn_status attn_lse_combine(const float* part_out, const float* part_lse, int n
     const long long blocks = (rows + 7) / 8;
     if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+    const unsigned g = static_cast<unsigned>(blocks);
     switch (D) {
-        case 32: attn::lse_combine_kernel<32><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
-        case 64: attn::lse_combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
-        case 128: attn::lse_combine_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
-        default: attn::lse_combine_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(part_out, part_lse, num_splits, rows, o, lse); break;
+        case 32: attn::lse_combine_kernel<32><<<g, 256, 0, stream>>>(part_out, part_lse, num_splits, rows, H, Tq, o, so.b, so.h, so.t, lse); break;
+        case 64: attn::lse_combine_kernel<64><<<g, 256, 0, stream>>>(part_out, part_lse, num_splits, rows, H, Tq, o, so.b, so.h, so.t, lse); break;
+        case 128: attn::lse_combine_kernel<128><<<g, 256, 0, stream>>>(part_out, part_lse, num_splits, rows, H, Tq, o, so.b, so.h, so.t, lse); break;
+        default: attn::lse_combine_kernel<256><<<g, 256, 0, stream>>>(part_out, part_lse, num_splits, rows, H, Tq, o, so.b, so.h, so.t, lse); break;
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     return ATTN_OK;
+}
+
+attn_status attn_lse_combine(const float* part_out, const float* part_lse, int num_splits, void* out, float* lse,
+                             int B, int H, int Tq, int D, cudaStream_t stream) {
+    return attn_lse_combine_strided(part_out, part_lse, num_splits, out, lse, B, H, Tq, D, nullptr, stream);
 }
 
 attn_status attn_get_device_status(cudaStream_t stream) {

@@ -90,6 +90,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     const int split = SPLIT ? unit % p.num_splits : 0;
     const int bh = SPLIT ? unit / p.num_splits : unit;
     const int b = bh / p.H;
+    const int h = bh - b * p.H;
     const int q0 = ptile * (2 * C::ROWS) + static_cast<int>(rank) * C::ROWS;
 
     int kv = __ldg(p.kv_len + b);
@@ -141,7 +142,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             const uint32_t lq = mapa_shared(PBAR(PB_Q), 0);
 #pragma unroll
             for (int blk = 0; blk < C::NBLK; ++blk)
-                tma_load_3d_pair(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, bh, lq);
+                tma_load_4d_pair(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, h, b, lq);
             int slot = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -158,13 +159,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < C::NBLK; ++c)
                         if (!(drop && c == 0))
-                            tma_load_3d_pair(dst + c * C::KBLK_BYTES, &tm_k, c * 64, key0 + static_cast<int>(rank) * C::KH,
-                                             bh, lfull);
+                            tma_load_4d_pair(dst + c * C::KBLK_BYTES, &tm_k, c * 64, key0 + static_cast<int>(rank) * C::KH,
+                                             h, b, lfull);
                 } else {
 #pragma unroll
                     for (int c = 0; c < C::NBLK / 2; ++c)
-                        tma_load_3d_pair(dst + c * C::VBLK_BYTES, &tm_v, static_cast<int>(rank) * (D / 2) + c * 64,
-                                         key0, bh, lfull);
+                        tma_load_4d_pair(dst + c * C::VBLK_BYTES, &tm_v, static_cast<int>(rank) * (D / 2) + c * 64,
+                                         key0, h, b, lfull);
                 }
                 if (++slot == C::NSLOTS) {
                     slot = 0;
@@ -415,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                     *reinterpret_cast<float4*>(dst + e) = v4;
                 }
             } else {
-                __nv_bfloat16* dst = p.out + (static_cast<long long>(bh) * p.Tq + row) * D + oc * 32;
+                __nv_bfloat16* dst = p.out + b * p.out_sb + h * p.out_sh + row * p.out_st + oc * 32;
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint4 v4;

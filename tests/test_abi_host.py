@@ -152,3 +152,26 @@ def test_segments_geometry_and_argument_checks(lib):
     assert f(A, A, A, A, A, 2, NULL, A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1    # no workspace
     assert f(A, A, A, A, A, 2, ctypes.c_void_p(0x10004), A, NULL, 1, 1, 8, 8, 64, 0.1, NULL) == 1
     assert f(A, A, A, A, A, 2, A, A, NULL, 1, 1, 8, 8, 96, 0.1, NULL) == 2       # head dim
+
+
+class _Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("t", ctypes.c_int64)]
+
+
+def test_strided_entries_check_strides(lib):
+    f = lib.attn_prefix_fwd_strided
+    ok = _Strides(8 * 64 * 64, 64, 8 * 64)          # a [B,T,H,D] layout with H=8, D=64
+    bad_align = _Strides(8 * 64 * 64, 60, 8 * 64)   # h stride not a multiple of 8
+    bad_row = _Strides(8 * 64 * 64, 64, 32)         # t stride shorter than a row
+    neg = _Strides(-8, 64, 8 * 64)
+    for s in (bad_align, bad_row, neg):
+        for pos in range(4):
+            args = [NULL] * 4
+            args[pos] = ctypes.c_void_p(ctypes.addressof(s))
+            assert f(A, A, A, A, A, NULL, 1, 8, 8, 8, 64, 0.1, *args, NULL) == 1
+    del ok
+    g = lib.attn_prefix_fwd_split_strided
+    assert g(A, A, A, A, 4, A, A, 1, 8, 8, 8, 64, 0.1, ctypes.c_void_p(ctypes.addressof(bad_row)),
+             NULL, NULL, NULL) == 1
+    c = lib.attn_lse_combine_strided
+    assert c(A, A, 4, A, NULL, 1, 8, 8, 64, ctypes.c_void_p(ctypes.addressof(bad_align)), NULL) == 1
