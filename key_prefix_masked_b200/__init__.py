@@ -10,6 +10,7 @@ int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never tak
 The computation runs in the hand-written kernels of the C library built from csrc/;
 this package only marshals arguments.
 """
+from . import sharded  # noqa: F401  (key-sharded attention across ranks)
 from ._binding import (  # noqa: F401
     AttnError,
     ATTN_OK,
