@@ -174,32 +174,6 @@ __device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity,
     return true;
 }
 
-// Cluster-scope variants for barriers completed by the other CTA of a pair.
-__device__ __noinline__ bool wait_bar_cl(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned long long limit_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            atomicOr(&g_attn_status, STATUS_TIMEOUT);
-            return false;
-        }
-    }
-}
-__device__ __noinline__ bool wait_bar_drain_cl(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait_cluster(bar, parity)) {
-        if (global_timer_ns() - t0 > limit_ns) {
-            atomicOr(&g_attn_status, STATUS_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
 // Exact combination of one row's split partials, by one warp (lane = thread % 32):
 //   M = max_c lse_c,  lse = M + ln sum_c exp(lse_c - M),  out = sum_c exp(lse_c - lse) O_c,
 // the log-sum-exp rule of split-KV; a row whose every chunk is empty gives 0 / -inf.

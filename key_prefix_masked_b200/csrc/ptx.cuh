@@ -59,16 +59,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ void tma_prefetch_map(const void* map) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// 3-D tiled bulk-tensor copy global -> shared, completing on an mbarrier (tx bytes).
-// x (innermost coordinate) must be a multiple of 8 elements for 16-bit data.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, int x, int y, int z,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
 // 4-D tiled TMA load (coordinates innermost first), completing on `bar`.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, int x, int y, int z, int w,
                                             uint32_t bar) {
@@ -77,11 +67,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, int x
         " [%0], [%1, {%2, %3, %4, %5}], [%6];\n" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
         : "memory");
-}
-// Orders this thread's generic-proxy shared-memory writes before later async-proxy
-// (TMA / tensor-core) accesses.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -185,45 +170,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-// Phase probe with cluster-scope acquire (for barriers that other CTAs' threads,
-// copies or commits complete).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n"
-        ".reg .pred p;\n"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        "selp.u32 %0, 1, 0, p;\n"
-        "}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 // Arrival on an mbarrier in another CTA of the cluster (default semantics: release at
 // CTA scope, the form the CUDA pair pipelines use for cross-CTA handshakes).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
-// Atomic add with cluster-scope release on a word in (possibly another CTA's) shared memory.
-__device__ __forceinline__ void red_add_release_cluster(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;\n" ::"r"(cluster_addr), "r"(v) : "memory");
-}
 __device__ __forceinline__ uint32_t ld_acquire_cluster_smem(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
     return v;
-}
-// 3-D tiled copy issued by either CTA of a pair into its own shared memory, completing
-// the transaction bytes on the mbarrier at `bar_cluster` (a shared::cluster address,
-// here always the leader CTA's barrier).
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* map, int x, int y, int z,
-                                                 uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
-        : "memory");
 }
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* map, int x, int y, int z, int w,
                                                  uint32_t bar_cluster) {

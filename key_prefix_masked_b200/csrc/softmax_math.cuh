@@ -1,7 +1,7 @@
 // softmax_math.cuh -- packed fp32 arithmetic of sm_100 for the softmax warps.
 //
 // Blackwell executes two fp32 FMAs or adds in one instruction (fma.rn.f32x2,
-// add.rn.f32x2, mul.rn.f32x2 on a 64-bit register pair) and takes the maximum of
+// add.rn.f32x2 on a 64-bit register pair) and takes the maximum of
 // three operands in one instruction (max.f32 with three sources).  The softmax of a
 // 128-column row spends most of its issue slots on exactly these operations, so using
 // them halves the instruction count of the max, scale-and-shift and row-sum steps.
@@ -30,16 +30,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
         "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
