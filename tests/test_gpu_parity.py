@@ -59,6 +59,10 @@ SWEEP = [
     (1, 1, 1, 17, (16,)),
     (2, 1, 256, 640, (15, 17)),
     (1, 1, 383, 130, (130,)),
+    (1, 1, 1, 1, (1,)),                       # one query, one key
+    (1, 2, 1, 1000, (1000,)),                 # one query row against a long prefix
+    (4, 16, 33, 65, (65, 1, 64, 0)),          # many (b, h) slices of short sequences
+    (1, 1, 513, 1024, (1024,)),               # a CTA pair whose second tile holds one row
 ]
 
 
@@ -226,6 +230,14 @@ def test_workload_ragged(kp):
 
 def test_workload_splitkv(kp):
     _workload_check(kp, "splitkv", n_random=0, splits=64)
+
+
+def test_workload_unmasked_8v(kp):
+    _workload_check(kp, "unmasked_8v", n_random=24)
+
+
+def test_workload_unmasked_32v(kp):
+    _workload_check(kp, "unmasked_32v", n_random=24)
 
 
 def test_workload_unmasked_d128(kp):
