@@ -222,8 +222,8 @@ void attn_set_wait_limit_ns(uint64_t ns);
  * announce one key-tile copy without issuing it, so that the consumer's bounded wait
  * runs out (exercises the ATTN_ERR_TIMEOUT path without faulting anything).  0 = off. */
 #define ATTN_DEBUG_DROP_COPY 1u
-/* Test hook: run head dim 256 on the single-CTA kernel instead of the CTA-pair kernel
- * (for side-by-side checks of the two implementations). */
+/* Test hook: run head dims 128 and 256 on the single-CTA kernel instead of the CTA-pair
+ * kernel (for side-by-side checks of the two implementations). */
 #define ATTN_DEBUG_SINGLE_CTA 2u
 void attn_set_debug_flags(unsigned flags);
 

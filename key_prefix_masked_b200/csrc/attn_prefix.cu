@@ -1021,11 +1021,12 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, const Stride
     return ATTN_OK;
 }
 
-// Head dim 256 runs on CTA pairs: 256-row query tiles, each CTA copying half of K and V.
-template <bool SPLIT>
+// Head dims 128 and 256 run on CTA pairs: 256-row query tiles, each CTA copying half of
+// K and V.
+template <int D, bool SPLIT>
 attn_status launch_fwd_pair(const void* q, const void* k, const void* v, const Strides* st, Params prm,
                             cudaStream_t stream) {
-    using C = attn::PairCfg;
+    using C = attn::PairCfg<D>;
     const long long BH = static_cast<long long>(prm.B) * prm.H;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, prm.B, prm.H, prm.Tq, C::D, st[0], 64, C::ROWS, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1035,7 +1036,7 @@ attn_status launch_fwd_pair(const void* q, const void* k, const void* v, const S
     prm.n_qtiles = (prm.Tq + 2 * C::ROWS - 1) / (2 * C::ROWS);
     const long long grid = 2LL * prm.n_qtiles * BH * (SPLIT ? prm.num_splits : 1);
     if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    auto kern = attn::attn_fwd_pair_kernel<SPLIT>;
+    auto kern = attn::attn_fwd_pair_kernel<D, SPLIT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
@@ -1054,10 +1055,12 @@ attn_status dispatch_fwd(int D, const void* q, const void* k, const void* v, con
     switch (D) {
         case 32: return launch_fwd<32, SPLIT>(q, k, v, st, prm, stream);
         case 64: return launch_fwd<64, SPLIT>(q, k, v, st, prm, stream);
-        case 128: return launch_fwd<128, SPLIT>(q, k, v, st, prm, stream);
+        case 128:
+            if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<128, SPLIT>(q, k, v, st, prm, stream);
+            return launch_fwd_pair<128, SPLIT>(q, k, v, st, prm, stream);
         case 256:
             if (prm.debug & ATTN_DEBUG_SINGLE_CTA) return launch_fwd<256, SPLIT>(q, k, v, st, prm, stream);
-            return launch_fwd_pair<SPLIT>(q, k, v, st, prm, stream);
+            return launch_fwd_pair<256, SPLIT>(q, k, v, st, prm, stream);
         default: return ATTN_ERR_UNSUPPORTED;
     }
 }

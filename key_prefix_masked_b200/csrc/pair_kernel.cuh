@@ -1,13 +1,14 @@
-// pair_kernel.cuh -- head-dim-256 forward on a CTA pair (cta_group::2).  Included by
-// attn_prefix.cu inside namespace attn, after the single-CTA kernel's helpers.
+// pair_kernel.cuh -- forward on a CTA pair (cta_group::2) for head dims 128 and 256.
+// Included by attn_prefix.cu inside namespace attn, after the single-CTA kernel's helpers.
 //
 // A cluster of two CTAs shares one 256-row query tile: each CTA holds its own 128 query
 // rows (Q in its shared memory, S / P / O in its TMEM lanes) and HALF of every key and
-// value tile -- keys [64r, 64r + 64) of K, value columns [128r, 128r + 128) of V for
+// value tile -- keys [64r, 64r + 64) of K, value columns [r*D/2, (r+1)*D/2) of V for
 // CTA rank r.  The leader CTA's single MMA thread issues M = 256 tcgen05 MMAs that read
-// A from each CTA and B split across both, so each CTA streams 64 KB of K/V per 128-key
-// tile instead of 128 KB: the five 32 KB ring slots hold 2.5 tiles of look-ahead, which
-// takes the copy latency off the critical path.
+// A from each CTA and B split across both, so each CTA streams half of every K/V tile
+// (64 KB at D=256, 32 KB at D=128) and the MMA thread issues one instruction per 256
+// rows: at D=256 the five 32 KB ring slots hold 2.5 tiles of look-ahead, at D=128 twelve
+// 16 KB slots hold 6.
 //
 // Roles (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
 // producer (both CTAs, into their own memory, completing on the leader's barriers);
@@ -23,42 +24,48 @@
 // the columns that belong to earlier tiles or ranges are masked by selection, so key
 // padding is never read.
 
+constexpr int PAIR_MAX_SLOTS = 12;
+
+template <int D_>
 struct PairCfg {
-    static constexpr int D = 256;
+    static constexpr int D = D_;
     static constexpr int ROWS = 128;                 // query rows per CTA (TMEM lanes)
     static constexpr int NBLK = D / 64;              // 64-column (128-byte) blocks per row
-    static constexpr int Q_BYTES = ROWS * D * 2;     // 64 KB
+    static constexpr int Q_BYTES = ROWS * D * 2;     // 64 KB at D=256
     static constexpr int KH = BN / 2;                // keys of a K tile held by one CTA
     static constexpr int KBLK_BYTES = KH * 128;      // one 64-column block of them: 8 KB
     static constexpr int VBLK_BYTES = BN * 128;      // one 64-column block of V: 16 KB
-    static constexpr int SLOT = 32768;               // one CTA's half of a K or V tile
+    static constexpr int SLOT = NBLK * KBLK_BYTES;   // one CTA's half of a K or V tile
     static constexpr int CTRL = 1024;
-    static constexpr int NSLOTS = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
+    static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
+    static constexpr int NSLOTS = NSLOTS_FIT < PAIR_MAX_SLOTS ? NSLOTS_FIT : PAIR_MAX_SLOTS;
     static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
     static constexpr int THREADS = 224;
-    static_assert(NSLOTS >= 4 && NSLOTS <= 8, "pair ring depth");
+    static_assert(D == 128 || D == 256, "pair head dims");
+    static_assert(NSLOTS >= 4, "pair ring depth");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "pair shared memory budget");
-    static_assert(NBLK * KBLK_BYTES == SLOT && (NBLK / 2) * VBLK_BYTES == SLOT, "half tiles fill a slot");
+    static_assert((NBLK / 2) * VBLK_BYTES == SLOT, "a V half fills a slot like a K half");
+    static_assert(O_COL + D <= TMEM_COLS, "pair TMEM budget");
 };
 
 enum : int {
     PB_Q = 0,
-    PB_FULL = 1,     // [8] slot filled by both CTAs' copies (leader)
-    PB_EMPTY = 9,    // [8] slot consumed (multicast commit, both CTAs)
-    PB_S = 17,       // [2] S_j ready (multicast commit, both CTAs)
-    PB_OLAST = 19,   // PV_{n-1} complete (multicast commit, both CTAs; completes once)
-    PB_DRAIN = 20,   // leader only
-    PB_P = 21,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
-    PB_OPREV = 23,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
-    PB_NUM = 24
+    PB_FULL = 1,     // [PAIR_MAX_SLOTS] slot filled by both CTAs' copies (leader)
+    PB_EMPTY = 13,   // [PAIR_MAX_SLOTS] slot consumed (multicast commit, both CTAs)
+    PB_S = 25,       // [2] S_j ready (multicast commit, both CTAs)
+    PB_OLAST = 27,   // PV_{n-1} complete (multicast commit, both CTAs; completes once)
+    PB_DRAIN = 28,   // leader only
+    PB_P = 29,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
+    PB_OPREV = 31,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
+    PB_NUM = 32
 };
+static_assert(PB_EMPTY == PB_FULL + PAIR_MAX_SLOTS && PB_S == PB_EMPTY + PAIR_MAX_SLOTS, "pair barrier map");
 
-template <bool SPLIT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+template <int D, bool SPLIT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    using C = PairCfg;
-    constexpr int D = C::D;
+    using C = PairCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     // Swizzled tiles need 1024-byte alignment; both CTAs see the same layout, so both
     // return here together (no cluster barrier has been reached yet).

@@ -1,6 +1,6 @@
-"""Head dim 256 has two implementations: CTA pairs (default) and a single-CTA kernel
-(selected by the ATTN_DEBUG_SINGLE_CTA test hook).  Both must match the oracle and
-each other, single pass and split."""
+"""Head dims 128 and 256 have two implementations: CTA pairs (default) and a single-CTA
+kernel (selected by the ATTN_DEBUG_SINGLE_CTA test hook).  Both must match the oracle
+and each other, single pass and split."""
 import numpy as np
 import pytest
 import torch
@@ -23,14 +23,15 @@ def kp():
 SINGLE_CTA = 2
 
 
+@pytest.mark.parametrize("D", [128, 256])
 @pytest.mark.parametrize("shape", [
     (2, 2, 300, 700, (700, 129)),
     (1, 3, 513, 1000, (999,)),
     (3, 1, 130, 256, (0, 1, 255)),
 ])
-def test_pair_and_single_cta_agree(kp, shape):
+def test_pair_and_single_cta_agree(kp, D, shape):
     B, H, Tq, Tk, lens = shape
-    c = synth.random_case(B, H, Tq, Tk, 256, lens, seed=Tq)
+    c = synth.random_case(B, H, Tq, Tk, D, lens, seed=Tq + D)
     g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in c.items()}
     kp.set_debug_flags(0)
     o_pair, l_pair = kp.attn_prefix_fwd(g["q"], g["k"], g["v"], g["kv_len"])

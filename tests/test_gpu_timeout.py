@@ -23,7 +23,7 @@ def kp():
     kp.set_wait_limit_ns(1_000_000_000)
 
 
-@pytest.mark.parametrize("D,flags", [(256, 0), (256, SINGLE_CTA), (64, 0), (128, 0)])
+@pytest.mark.parametrize("D,flags", [(256, 0), (256, SINGLE_CTA), (64, 0), (128, 0), (128, SINGLE_CTA)])
 def test_dropped_copy_times_out_and_context_survives(kp, D, flags):
     import oracle
     c = synth.random_case(1, 2, 200, 500, D, (480,), seed=D + flags)
