@@ -620,15 +620,15 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         s_read(j + 1);
                         relay_s();
                     }
+                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();   // V_j first: usually landed
                     ok = ok && wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
-                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();
                     publish();
                 }
             } else {
 #pragma unroll 1
                 for (int j = 0; j < n_tiles && ok; ++j) {
-                    ok = wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
-                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();
+                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();   // V_j first: usually landed
+                    ok = ok && wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
                     publish();
                     if (j + 2 < n_tiles) relay_s();
                 }

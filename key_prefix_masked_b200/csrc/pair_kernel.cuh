@@ -41,6 +41,11 @@ struct PairCfg {
     static constexpr int NSLOTS = NSLOTS_FIT < PAIR_MAX_SLOTS ? NSLOTS_FIT : PAIR_MAX_SLOTS;
     static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
     static constexpr int THREADS = 224;
+    // Who waits for "P_j stored": at D=128 the MMA thread probes the P barrier itself
+    // (non-suspending test_wait), which takes the relay's wake-up off the P -> PV
+    // handshake; at D=256 the MMA thread has twice the MMAs to issue per tile and the
+    // relay keeps that wait (measured: +2 to +4 % at D=128, -1.5 % at D=256 the other way).
+    static constexpr bool MMA_WAITS_P = D <= 128;
     static_assert(D == 128 || D == 256, "pair head dims");
     static_assert(NSLOTS >= 4, "pair ring depth");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "pair shared memory budget");
@@ -198,8 +203,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
     } else if (warp == 6) {
         // ================================================================ wait relay (leader)
         // Waits on Q and, in the MMA thread's consumption order, on K_0, K_1, then per tile
-        // "P_j stored in both CTAs and V_j landed" and K_{j+2}; publishes the count of
-        // completed events with a release store.
+        // "V_j landed and P_j stored in both CTAs" (without P_j when the MMA thread probes
+        // it itself) and K_{j+2}; publishes the count of completed events with a release
+        // store.
         if (leader && lane == 0 && n_tiles > 0) {
             uint32_t seq = 0;
             bool ok = wait_bar(PBAR(PB_Q), 0, abort_flag, wlim);
@@ -224,8 +230,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             }
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
-                ok = wait_bar(PBAR(PB_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
-                item();  // V_j
+                item();  // V_j: waited first, as it has usually landed long before P_j, so
+                         // that "P_j stored" reaches the MMA thread one wait sooner
+                if constexpr (!C::MMA_WAITS_P)
+                    ok = ok && wait_bar(PBAR(PB_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
                 publish();
                 if (j + 2 < n_tiles) {
                     item();  // K_{j+2}
@@ -277,8 +285,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 next_slot();
             };
             auto issue_pv = [&](int j) {
-                ok = poll_ge(seq_addr, ++consumed);   // P_j stored in both CTAs and V_j halves landed
+                ok = poll_ge(seq_addr, ++consumed);   // V_j halves landed (and P_j stored, via the relay)
                 if (!ok) return;
+                if constexpr (C::MMA_WAITS_P) {
+                    // P_j stored in both CTAs: probed here, without suspending
+                    const uint32_t pb = PBAR(PB_P + (j & 1));
+                    const uint32_t par = (j >> 1) & 1;
+                    if (!mbar_test_wait(pb, par)) {
+                        const uint64_t t0 = global_timer_ns();
+                        while (!mbar_test_wait(pb, par)) {
+                            if (*abort_flag) {
+                                ok = false;
+                                return;
+                            }
+                            if (global_timer_ns() - t0 > wlim) {
+                                *abort_flag = 1;
+                                atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                                ok = false;
+                                return;
+                            }
+                        }
+                    }
+                }
                 tc_fence_after();
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
                 const uint64_t vd = slot_desc(v_desc0);
