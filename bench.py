@@ -289,9 +289,10 @@ def run_ours(args, rank, world):
     peaks, peaks_src = load_peaks()
     kern_avg_ms = statistics.mean(kern_ms)
     achieved = flops / (kern_avg_ms * 1e-3) / 1e12
-    # the dominant kernel: head dim 256 runs on CTA pairs, others on single CTAs
-    kernel_tag = "attn_fwd_pair" if w.D == 256 else f"attn_fwd_d{w.D}"
-    kernel_name = (f"attn_fwd_pair_kernel<{int(bool(splits))}>" if w.D == 256
+    # the dominant kernel: head dims 128 and 256 run on CTA pairs, 32 and 64 on single CTAs
+    pair = w.D in (128, 256)
+    kernel_tag = "attn_fwd_pair" if w.D == 256 else (f"attn_fwd_pair_d{w.D}" if pair else f"attn_fwd_d{w.D}")
+    kernel_name = (f"attn_fwd_pair_kernel<{w.D},{int(bool(splits))}>" if pair
                    else f"attn_fwd_kernel<{w.D},{int(bool(splits))}>")
     # A kernel that runs long enough to draw the power cap is compared with the sustained
     # cuBLAS figure; a short one (the D=64 shapes, ~1 ms steps) with the burst figure.
