@@ -10,22 +10,34 @@
 // log-sum-exp, so partial results over key chunks combine exactly ("Sequence-parallel
 // inference" on the same page): attn_prefix_fwd_split + attn_lse_combine.
 //
-// Kernel design (one CTA = one 128-row query tile of one (b, h), optionally one key
-// chunk; 6 warps):
-//   warp 4      TMA producer: Q tile once, then K and V chunks into a ring of 16 KB
-//               shared-memory slots, in exactly the order the MMA warp consumes them.
-//               Key tiles at or beyond kv_len are never requested.
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T with both operands in shared
-//               memory into a double-buffered fp32 TMEM tile (128 x 128), and
-//               O += P_j V_j with P read from TMEM (bf16, written over S_j) and V from
-//               shared memory into an fp32 TMEM accumulator (128 x D).  It also owns
-//               the TMEM allocation.
-//   warps 0-3   softmax + epilogue: thread t owns query row t (TMEM lane t).  Scores of
-//               keys >= kv_len are replaced by -inf by selection; the running max is
-//               kept in the log2 domain and O is rescaled in TMEM only when the max grows
-//               by more than 2^8 (exact either way: O and the row sum always share one
-//               reference max).  At the end O is divided by the row sum and written as
-//               bf16 (fp32 for split partials) with lse = ln(sum) + max.
+// Kernels in this file (the CTA-pair kernel for head dims 128 and 256 is in
+// pair_kernel.cuh, the multi-range key gather in segments.cuh):
+//
+// attn_fwd_kernel<D, SPLIT>: one CTA = one 128-row query tile of one (b, h), optionally
+// one key chunk.  Roles:
+//   producer warp   TMA: Q tile once, then K and V chunks into a ring of 16 KB shared-
+//                   memory slots, in exactly the order the MMA thread consumes them.  Key
+//                   tiles at or beyond kv_len are never requested.
+//   MMA warp        one thread: S_j = Q K_j^T with both operands in shared memory into a
+//                   double-buffered fp32 TMEM tile (128 x 128), and O += P_j V_j with P
+//                   read from TMEM and V from shared memory into an fp32 TMEM
+//                   accumulator (128 x D).  It also owns the TMEM allocation.
+//   relay warp      performs the blocking mbarrier waits in the MMA thread's order and
+//                   publishes a count of completed events, which the MMA thread polls.
+//   softmax warps   thread = query row = TMEM lane.  Scores of keys >= kv_len are
+//                   replaced by -inf by selection; the running max is kept in the log2
+//                   domain and O is rescaled in TMEM only when the max grows by more than
+//                   2^8 (exact either way: O and the row sum always share one reference
+//                   max).  At the end O is divided by the row sum and written as bf16
+//                   (fp32 for split partials) with lse = ln(sum) + max.
+// Head dims 32 and 64 run in two-group mode (two softmax warpgroups on alternate key
+// tiles, each with its own O accumulator and P buffer in TMEM, S issued ahead of PV,
+// turns at the exponentials, an exact log-sum-exp merge at the end; 352 threads).  Head
+// dims 128 and 256 (test hook only) use one softmax warpgroup that stores P over S (224
+// threads).
+// lse_combine_kernel<D>: the exact log-sum-exp combination of split partials, one warp
+// per output row (also run inside the split kernels when the combine is fused).
+//
 // The last, partial key tile of a range is read as the window [k_end - 128, k_end): every
 // row copied is a valid key (or a zero-filled row at a negative coordinate) and the
 // columns that belong to earlier tiles are masked by selection, so key padding (NaN
