@@ -125,10 +125,10 @@ def _check_qkv(q, k, v, kv_len, strided=False):
     B, H, Tq, D = q.shape
     if k.shape[:2] != (B, H) or k.shape[3] != D or v.shape != k.shape:
         raise ValueError("k and v must be [B,H,Tk,D] matching q's B, H, D")
-    if (not kv_len.is_cuda or kv_len.dtype != torch.int32 or kv_len.numel() != B
-            or not kv_len.is_contiguous()):
+    if kv_len is not None and (not kv_len.is_cuda or kv_len.dtype != torch.int32 or kv_len.numel() != B
+                               or not kv_len.is_contiguous()):
         raise ValueError("kv_len must be a contiguous int32 CUDA tensor of B entries")
-    if len({q.device, k.device, v.device, kv_len.device}) != 1:
+    if len({q.device, k.device, v.device} | ({kv_len.device} if kv_len is not None else set())) != 1:
         raise ValueError("all tensors must be on one device")
     return int(B), int(H), int(Tq), int(k.shape[2]), int(D)
 
@@ -275,8 +275,7 @@ def fwd_segments(q, k, v, seg_start, seg_len, scale=None, workspace=None, out=No
     if seg_start.shape != seg_len.shape:
         raise ValueError("seg_start and seg_len must have the same shape")
     S = int(seg_start.shape[1])
-    dummy_len = torch.zeros(B, dtype=torch.int32, device=q.device)
-    B, H, Tq, Tk, D = _check_qkv(q, k, v, dummy_len)
+    B, H, Tq, Tk, D = _check_qkv(q, k, v, None)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     need = int(lib().attn_segments_workspace_bytes(B, H, Tk, D))
     if workspace is None:
