@@ -246,3 +246,22 @@ def test_workload_unmasked_d128(kp):
 
 def test_workload_prefix_d128(kp):
     _workload_check(kp, "prefix_d128", n_random=16)
+
+
+@pytest.mark.parametrize("D", [64, 256])
+def test_grid_beyond_65535_slices(kp, D):
+    """131072 (b, h) slices of short sequences: a 1-D grid of more than 2^16 CTAs (and
+    CTA pairs at D=256), ragged kv_len drawn per element including 0."""
+    B, H, Tq, Tk = 512, 256, 8, 8
+    g = torch.Generator().manual_seed(170 + D)
+    lens = torch.randint(0, Tk + 1, (B,), generator=g).tolist()
+    case = synth.random_case(B, H, Tq, Tk, D, tuple(lens), seed=171 + D, device="cuda")
+    out, lse = kp.attn_prefix_fwd(case["q"], case["k"], case["v"], case["kv_len"], case["scale"])
+    torch.cuda.synchronize()
+    assert kp.device_status() == kp.ATTN_OK
+    bsel = [0, 1, 255, 256, 511]
+    q = case["q"][bsel].cpu()
+    k, v = case["k"][bsel].cpu(), case["v"][bsel].cpu()
+    ref_out, ref_lse = oracle.attn_prefix(q, k, v, [lens[b] for b in bsel], case["scale"])
+    assert_out_close(out[bsel], ref_out)
+    assert_lse_close(lse[bsel], ref_lse)
