@@ -265,3 +265,28 @@ def test_grid_beyond_65535_slices(kp, D):
     ref_out, ref_lse = oracle.attn_prefix(q, k, v, [lens[b] for b in bsel], case["scale"])
     assert_out_close(out[bsel], ref_out)
     assert_lse_close(lse[bsel], ref_lse)
+
+
+@pytest.mark.parametrize("D", [64, 256])
+def test_cuda_graph_capture_and_replay(kp, D):
+    """The forward captured into a CUDA graph (after one eager call) replays bit for bit;
+    new inputs copied into the captured buffers give the new result."""
+    c1 = synth.random_case(2, 2, 300, 700, D, (700, 129), seed=180 + D, device="cuda")
+    c2 = synth.random_case(2, 2, 300, 700, D, (64, 700), seed=181 + D, device="cuda")
+    q, k, v, kv = (c1[n].clone() for n in ("q", "k", "v", "kv_len"))
+    out = torch.empty_like(q)
+    lse = torch.empty(2, 2, 300, dtype=torch.float32, device="cuda")
+    kp.attn_prefix_fwd(q, k, v, kv, out=out, lse=lse)      # eager warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        kp.attn_prefix_fwd(q, k, v, kv, out=out, lse=lse)
+    for c in (c1, c2):
+        for dst, n in ((q, "q"), (k, "k"), (v, "v"), (kv, "kv_len")):
+            dst.copy_(c[n])
+        g.replay()
+        torch.cuda.synchronize()
+        ref_out, ref_lse = kp.attn_prefix_fwd(c["q"], c["k"], c["v"], c["kv_len"])
+        torch.cuda.synchronize()
+        assert bits_equal(out, ref_out) and bits_equal(lse, ref_lse)
+    assert kp.device_status() == kp.ATTN_OK
