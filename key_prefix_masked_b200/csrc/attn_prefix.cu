@@ -991,7 +991,6 @@ attn_status check_device() {
     return cached[dev] ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
-// 3-D map over a [B*H, T, D] bf16 tensor; box = (swizzle block columns, rows, 1).
 // A [B, H, T, D] bf16 tensor at element strides s (d contiguous) as a 4-D TMA map with
 // dims (D, T, H, B); a box is box_rows rows x box_cols columns of one (b, h).
 bool make_map(CUtensorMap* map, const void* base, int B, int H, int T, int D, const Strides& s, int box_cols,
