@@ -8,16 +8,29 @@
 // A from each CTA and B split across both, so each CTA streams half of every K/V tile
 // (64 KB at D=256, 32 KB at D=128) and the MMA thread issues one instruction per 256
 // rows: at D=256 the five 32 KB ring slots hold 2.5 tiles of look-ahead, at D=128 twelve
-// 16 KB slots hold 6.
+// 16 KB slots hold 6.  MMA order: S_0, S_1, then PV_j, S_{j+2} per tile j; P_j is stored
+// over S_j, and S_{j+2} overwrites it only after PV_j has read it (one thread's MMAs run
+// in issue order).
 //
-// Roles (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
-// producer (both CTAs, into their own memory, completing on the leader's barriers);
+// Roles at D=256 (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4
+// copy producer (both CTAs, into their own memory, completing on the leader's barriers);
 // warp 5 TMEM allocation (both) and MMA issue (leader); warp 6 wait relay (leader).
+// At D=128 the kernel runs in two-group mode (352 threads: softmax warps 0-7, then the
+// same three roles): warpgroup w takes the key tiles j = w (mod 2) with its own running
+// max, row sum and TMEM O accumulator O_w (S_0, S_1, O_0, O_1 fill the 512 columns), so
+// one group's softmax overlaps the other's P -> PV -> S round trip; the warps that share
+// a sub-partition take turns at the exponentials; the two partial results are merged
+// exactly at the end by the log-sum-exp rule of split-KV ("Sequence-parallel inference"
+// of "Add sequence-parallel multi-GPU inference ... and a cuDNN flash attention option").
+// S_j is issued after PV_{j-2}, the last PV into O_{j&1} before tile j, so "S_j ready"
+// already means that accumulator is quiescent and the group rescales it without waiting.
+//
 // Each softmax warp of either CTA announces P with one arrival on the leader's P
 // barrier (the remote mbarrier arrive with default semantics -- release at CTA scope --
 // which is the cross-CTA handshake the pair pipelines are built on; a cluster-scope
 // release costs ~450-1100 cycles and made this handshake the critical path).  The relay
-// folds "P_j stored in both CTAs" and "V_j landed" into one event for the MMA thread.
+// folds "P_j stored in both CTAs" and "V_j landed" into one event for the MMA thread
+// (at D=128 the MMA thread probes "P_j stored" itself).
 //
 // The last, partial key tile of a range is read as the window [k_end - 128, k_end):
 // every row copied is a valid key (or a zero-filled row at a negative coordinate), and
@@ -36,11 +49,19 @@ struct PairCfg {
     static constexpr int KBLK_BYTES = KH * 128;      // one 64-column block of them: 8 KB
     static constexpr int VBLK_BYTES = BN * 128;      // one 64-column block of V: 16 KB
     static constexpr int SLOT = NBLK * KBLK_BYTES;   // one CTA's half of a K or V tile
+    // Two-group mode (head dim 128): two softmax warpgroups on alternate key tiles, each
+    // with its own O accumulator; S_0, S_1, O_0, O_1 fill the 512 TMEM columns.
+    static constexpr bool DUAL = O_COL + 2 * D <= TMEM_COLS;
+    static constexpr int SM_WARPS = DUAL ? 8 : 4;    // softmax warps
+    static constexpr int WARP_PROD = SM_WARPS;       // copy producer (both CTAs)
+    static constexpr int WARP_MMA = SM_WARPS + 1;    // TMEM owner (both), MMA issuer (leader)
+    static constexpr int WARP_RELAY = SM_WARPS + 2;  // wait relay (leader)
+    static constexpr int THREADS = 32 * (SM_WARPS + 3);
     static constexpr int CTRL = 1024;
-    static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
+    static constexpr int XCH_BYTES = DUAL ? 2 * 2 * ROWS * 4 : 0;   // per-group (max, sum) exchange
+    static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL - XCH_BYTES) / SLOT;
     static constexpr int NSLOTS = NSLOTS_FIT < PAIR_MAX_SLOTS ? NSLOTS_FIT : PAIR_MAX_SLOTS;
-    static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
-    static constexpr int THREADS = 224;
+    static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL + XCH_BYTES;
     // Who waits for "P_j stored": at D=128 the MMA thread probes the P barrier itself
     // (non-suspending test_wait), which takes the relay's wake-up off the P -> PV
     // handshake; at D=256 the MMA thread has twice the MMAs to issue per tile and the
@@ -48,7 +69,7 @@ struct PairCfg {
     static constexpr bool MMA_WAITS_P = D <= 128;
     static_assert(D == 128 || D == 256, "pair head dims");
     static_assert(NSLOTS >= 4, "pair ring depth");
-    static_assert(SMEM_BYTES <= SMEM_LIMIT, "pair shared memory budget");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT && 2 * SMEM_BYTES > SMEM_LIMIT, "one CTA per SM, within budget");
     static_assert((NBLK / 2) * VBLK_BYTES == SLOT, "a V half fills a slot like a K half");
     static_assert(O_COL + D <= TMEM_COLS, "pair TMEM budget");
 };
@@ -62,7 +83,9 @@ enum : int {
     PB_DRAIN = 28,   // leader only
     PB_P = 29,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
     PB_OPREV = 31,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
-    PB_NUM = 32
+    PB_TURN = 32,    // [2][4] two-group mode: warp k of the group taking tile j may run its
+                     // exponentials (local; one arrival, by warp k of the other group)
+    PB_NUM = 40
 };
 static_assert(PB_EMPTY == PB_FULL + PAIR_MAX_SLOTS && PB_S == PB_EMPTY + PAIR_MAX_SLOTS, "pair barrier map");
 
@@ -130,11 +153,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
         mbar_init(PBAR(PB_DRAIN), 1);
         mbar_init(PBAR(PB_P + 0), 8);
         mbar_init(PBAR(PB_P + 1), 8);
+        for (int i = 0; i < 8; ++i) mbar_init(PBAR(PB_TURN + i), 1);
         words[1] = 0u;
         words[2] = 0u;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tmem_alloc_pair(smem_u32(words), TMEM_COLS);
         tmem_relinquish_pair();
     }
@@ -144,7 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
     const uint32_t tmem = words[0];
     const unsigned long long wlim = p.wait_ns;
 
-    if (warp == 4) {
+    if (warp == C::WARP_PROD) {
         // ================================================================ producer (both CTAs)
         if (lane == 0 && n_tiles > 0) {
             tma_prefetch_map(&tm_q);
@@ -200,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             }
         }
         __syncwarp();
-    } else if (warp == 6) {
+    } else if (warp == C::WARP_RELAY) {
         // ================================================================ wait relay (leader)
         // Waits on Q and, in the MMA thread's consumption order, on K_0, K_1, then per tile
         // "V_j landed and P_j stored in both CTAs" (without P_j when the MMA thread probes
@@ -242,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == C::WARP_MMA) {
         // ================================================================ MMA issuer (leader)
         if (leader && lane == 0 && n_tiles > 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(2 * C::ROWS, BN, false);
@@ -308,17 +332,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     }
                 }
                 tc_fence_after();
+                // PV_j reads P_j (over S_j); two-group mode: it adds into O_{j&1}, and
+                // each accumulator starts fresh
                 const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+                const uint32_t o_tmem = tmem + O_COL + (C::DUAL ? static_cast<uint32_t>((j & 1) * D) : 0u);
+                const uint32_t acc0 = (j < (C::DUAL ? 2 : 1)) ? 0u : 1u;
                 const uint64_t vd = slot_desc(v_desc0);
 #pragma unroll
                 for (int kb = 0; kb < BN / 16; ++kb)
-                    mma_ts_pair(tmem + O_COL, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV,
-                                (j == 0 && kb == 0) ? 0u : 1u);
+                    mma_ts_pair(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV, kb == 0 ? acc0 : 1u);
                 tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
                 // Each O barrier completes exactly once, so a parity-0 wait on it cannot
                 // be confused by a later phase.
-                if (j == n_tiles - 2) tc_commit_pair(PBAR(PB_OPREV), 0x3);
+                if (!C::DUAL && j == n_tiles - 2) tc_commit_pair(PBAR(PB_OPREV), 0x3);
                 if (j == n_tiles - 1) tc_commit_pair(PBAR(PB_OLAST), 0x3);
                 next_slot();
             };
@@ -333,16 +360,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             wait_bar_drain(PBAR(PB_DRAIN), 0, wlim);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < C::SM_WARPS) {
         // ================================================================ softmax (both CTAs)
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // Thread t of warpgroup w owns query row q0 + t % 128 (TMEM lane t % 128).  Two-group
+        // mode: group w takes the key tiles j = w (mod 2) with its own running max, row sum
+        // and O accumulator O_w, and the two partial results are merged exactly at the end
+        // (the log-sum-exp rule of split-KV); otherwise group 0 takes every tile.
+        constexpr bool DUAL = C::DUAL;
+        const int wg = warp >> 2;
+        const int r = tid & 127;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t o_col = O_COL + (DUAL ? static_cast<uint32_t>(wg * D) : 0u);
         const float sl2 = p.scale_log2;
         const bool pos_scale = sl2 > 0.0f;
         float m_ref = -INFINITY;
         float l_sum = 0.0f;
         bool ok = true;
+        int seen = 0;   // tiles this group has processed
 #pragma unroll 1
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int j = DUAL ? wg : 0; j < n_tiles; j += DUAL ? 2 : 1) {
+            // Two-group mode: S_j was issued after PV_{j-2}, the last PV into O_w before
+            // this tile, and its commit completes after every earlier MMA: from here on O_w
+            // is quiescent until PV_j, which needs this tile's P.
             ok = __all_sync(0xffffffffu, wait_bar(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
@@ -365,7 +404,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             const float mx = row_max(x) * (pos_scale ? sl2 : 1.0f);   // three-input maxima
             float factor = 1.0f;
             bool rescale = false;
-            if (j == 0) {
+            if (seen == 0) {
                 m_ref = mx;
             } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
                 const float m_new = fmaxf(m_ref, mx);
@@ -375,6 +414,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             }
             const float mul = pos_scale ? sl2 : 1.0f;
             const float neg_m = -m_ref;
+            if constexpr (DUAL) {
+                // Turns at the exponentials, in tile order, between the two warps of this
+                // CTA that share a sub-partition (and so its MUFU): warp k of each group.
+                if (j >= 1) {
+                    ok = __all_sync(0xffffffffu, wait_bar(PBAR(PB_TURN + (j & 1) * 4 + (warp & 3)),
+                                                          ((j - 1) >> 1) & 1, abort_flag, wlim));
+                    if (!ok) break;
+                }
+            }
             // p = 2^(x * mul - m): the scale-and-shift and the row sum in packed pairs
             float2 sp[4];
 #pragma unroll
@@ -394,30 +442,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 }
                 tmem_st16(s_addr + cc * 16, pk);
             }
+            if constexpr (DUAL) {
+                if (j + 1 < n_tiles) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(PBAR(PB_TURN + ((j + 1) & 1) * 4 + (warp & 3)));
+                }
+            }
             const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
             l_sum = l_sum * factor + tile_sum;
             if (rescale) {
-                // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last tile
-                // the leader announces PV_{n-2} on its own barrier.
-                const bool w = (j + 1 < n_tiles)
-                                   ? wait_bar(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
-                                   : wait_bar(PBAR(PB_OPREV), 0, abort_flag, wlim);
-                ok = __all_sync(0xffffffffu, w);
-                if (!ok) break;
-                tc_fence_after();
+                if constexpr (!DUAL) {
+                    // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last
+                    // tile the leader announces PV_{n-2} on its own barrier.
+                    const bool w = (j + 1 < n_tiles)
+                                       ? wait_bar(PBAR(PB_S + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, wlim)
+                                       : wait_bar(PBAR(PB_OPREV), 0, abort_flag, wlim);
+                    ok = __all_sync(0xffffffffu, w);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
 #pragma unroll 1
                 for (int oc = 0; oc < D / 32; ++oc) {
                     uint32_t o[32];
-                    tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+                    tmem_ld32_wait(tmem + lane_base + o_col + oc * 32, o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                    tmem_st32(tmem + lane_base + O_COL + oc * 32, o);
+                    tmem_st32(tmem + lane_base + o_col + oc * 32, o);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(mapa_shared(PBAR(PB_P + (j & 1)), 0));
+            ++seen;
         }
         // ---- epilogue
         if (ok && n_tiles > 0) {
@@ -426,20 +483,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }
-        const int row = q0 + tid;
+        // Two-group mode: m = max_w m_w, f_w = 2^(m_w - m), l = sum_w l_w f_w,
+        // O = sum_w O_w f_w / l (a group with no tile has l_w = 0 and weight 0).
+        float f_own = 1.0f, f_other = 0.0f, m_row = m_ref, l_row = l_sum;
+        bool own_has = n_tiles > 0, other_has = false;
+        if constexpr (DUAL) {
+            float* xch = reinterpret_cast<float*>(sKV + C::NSLOTS * C::SLOT + C::CTRL);   // [2][max, sum][128]
+            xch[(wg * 2 + 0) * 128 + r] = m_ref;
+            xch[(wg * 2 + 1) * 128 + r] = l_sum;
+            named_barrier_sync(XCH_ID, 32 * C::SM_WARPS);
+            const float m_o = xch[((wg ^ 1) * 2 + 0) * 128 + r];
+            const float l_o = xch[((wg ^ 1) * 2 + 1) * 128 + r];
+            own_has = l_sum > 0.0f;
+            other_has = l_o > 0.0f;
+            m_row = own_has ? (other_has ? fmaxf(m_ref, m_o) : m_ref) : m_o;
+            f_own = own_has ? fast_exp2(m_ref - m_row) : 0.0f;
+            f_other = other_has ? fast_exp2(m_o - m_row) : 0.0f;
+            l_row = l_sum * f_own + l_o * f_other;
+        }
+        const int row = q0 + r;
         const bool in_range = row < p.Tq;
         const bool have = n_tiles > 0;
-        const float inv_l = have ? 1.0f / l_sum : 0.0f;
-        const float lse_val = have ? (m_ref + log2f(l_sum)) * LN2 : -INFINITY;
+        const float inv_l = have ? 1.0f / l_row : 0.0f;
+        const float lse_val = have ? (m_row + log2f(l_row)) * LN2 : -INFINITY;
         const long long BH = static_cast<long long>(p.B) * p.H;
+        const uint32_t o_col_other = O_COL + static_cast<uint32_t>((wg ^ 1) * D);
+        // two-group mode: group w writes the 32-column chunks oc = w (mod 2)
 #pragma unroll 1
-        for (int oc = 0; oc < D / 32; ++oc) {
+        for (int oc = DUAL ? wg : 0; oc < D / 32; oc += DUAL ? 2 : 1) {
             uint32_t o[32];
-            if (have) {
-                tmem_ld32_wait(tmem + lane_base + O_COL + oc * 32, o);
+            if (have && own_has) {
+                tmem_ld32_wait(tmem + lane_base + o_col + oc * 32, o);
+                if constexpr (DUAL) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_own);
+                }
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            if (DUAL && have && other_has) {
+                uint32_t o2[32];
+                tmem_ld32_wait(tmem + lane_base + o_col_other + oc * 32, o2);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[e] = __float_as_uint(fmaf(__uint_as_float(o2[e]), f_other, __uint_as_float(o[e])));
             }
             if (!in_range) continue;
             if constexpr (SPLIT) {
@@ -463,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 }
             }
         }
-        if (in_range) {
+        if (in_range && wg == 0) {
             if constexpr (SPLIT) {
                 p.part_lse[(static_cast<long long>(split) * BH + bh) * p.Tq + row] = lse_val;
             } else if (p.lse != nullptr) {
@@ -476,7 +564,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
     // may still touch the other one.
     tc_fence_before();
     cluster_sync();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, TMEM_COLS);
     }
