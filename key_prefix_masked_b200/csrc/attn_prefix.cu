@@ -712,6 +712,17 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             const float mul = pos_scale ? sl2 : 1.0f;
             const float neg_m = -m_ref;
             if constexpr (DUAL) {
+                // PV_{j-2}, this group's previous PV, reads P_w and adds into O_w: it must be
+                // complete before P_w is rewritten (P is stored as it is computed, below) and
+                // before O_w is rescaled.  The parity wait is unambiguous: the barrier has
+                // passed the phase before (waited on this group's previous tile) and cannot
+                // pass the one after, whose PV needs this tile's P.
+                if (seen > 0) {
+                    ok = __all_sync(0xffffffffu,
+                                    wait_bar(BAR(BAR_PVD + (j & 1)), (seen - 1) & 1, abort_flag, wlim));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
                 // The groups take turns at the exponentials in tile order, so one group's
                 // MUFU-bound phase overlaps the other's loads, max and MMA round trip
                 // instead of both contending for the MUFU at once.  Group w waits on
@@ -722,49 +733,37 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     if (!ok) break;
                 }
             }
-            // p = 2^(x * mul - m).  One group: the scale-and-shift and the row sum in packed
-            // pairs.  Two-group mode keeps them scalar: its P is held in registers until
-            // the store, and the packed pairs' register alignment then costs spills.
+            // p = 2^(x * mul - m): the scale-and-shift and the row sum in packed pairs; P is
+            // stored 32 columns at a time, over S_j (one group) or into P_w (two groups).
+            const uint32_t p_addr = DUAL ? tmem + lane_base + C::P_COL + static_cast<uint32_t>(j & 1) * (BN / 2) : s_addr;
             float2 sp[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
             const float2 mul_2 = make_float2(mul, mul);
             const float2 neg_m2 = make_float2(neg_m, neg_m);
-            uint32_t pk[BN / 2];
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    float p0, p1;
-                    if constexpr (DUAL) {
-                        p0 = fast_exp2(fmaf(x[cc * 32 + 2 * e], mul, neg_m));
-                        p1 = fast_exp2(fmaf(x[cc * 32 + 2 * e + 1], mul, neg_m));
-                        if (e & 4) sp[e & 3].y += p0 + p1;
-                        else sp[e & 3].x += p0 + p1;
-                    } else {
-                        const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
-                        p0 = fast_exp2(y.x);
-                        p1 = fast_exp2(y.y);
-                        sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
-                    }
-                    pk[cc * 16 + e] = pack_bf16x2(p0, p1);
+                    const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
+                    const float p0 = fast_exp2(y.x);
+                    const float p1 = fast_exp2(y.y);
+                    sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
-                if constexpr (!DUAL) tmem_st16_at(s_addr + cc * 16, &pk[cc * 16]);   // P over S_j
+                tmem_st16_at(p_addr + cc * 16, pk);
             }
             if constexpr (DUAL) {
                 if (j + 1 < n_tiles) warp_arrive(BAR(BAR_TURN + ((j + 1) & 1)));
             }
             const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
             l_sum = l_sum * factor + tile_sum;
-            // This group's previous PV (PV_{j-2} in two-group mode, else PV_{j-1}) must be
-            // complete before O is rescaled, and (two-group mode) before P_w is rewritten.
-            // The parity wait is unambiguous: the barrier has passed the phase before
-            // (two-group mode: this group waited for it on its previous tile; one group:
-            // S_j, issued after PV_{j-2}, is complete) and cannot pass the one after, whose
-            // PV needs this tile's P.
-            if (seen > 0 && (DUAL || rescale)) {
-                ok = __all_sync(0xffffffffu,
-                                wait_bar(BAR(BAR_PVD + (DUAL ? (j & 1) : 0)), (seen - 1) & 1, abort_flag, wlim));
+            // One group: PV_{j-1} must be complete before O is rescaled.  The parity wait is
+            // unambiguous: S_j, issued after PV_{j-2}, is complete, so the barrier has passed
+            // the phase before; the phase after needs this tile's P.
+            if (!DUAL && seen > 0 && rescale) {
+                ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_PVD), (seen - 1) & 1, abort_flag, wlim));
                 if (!ok) break;
                 tc_fence_after();
             }
@@ -777,11 +776,6 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
                     tmem_st32(tmem + lane_base + o_col + oc * 32, o);
                 }
-            }
-            if constexpr (DUAL) {
-                const uint32_t p_addr = tmem + lane_base + C::P_COL + static_cast<uint32_t>(j & 1) * (BN / 2);
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) tmem_st16_at(p_addr + cc * 16, &pk[cc * 16]);
             }
             tmem_wait_st();
             warp_arrive(BAR(BAR_P + (j & 1)));
