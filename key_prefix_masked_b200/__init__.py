@@ -5,8 +5,11 @@
     out, lse = attn_prefix_fwd_split_fused(q, k, v, kv_len, num_splits=64)  # one launch
     out, lse = attn_prefix_fwd_segments(q, k, v, seg_start, seg_len)        # multi-range keys
 
-q, k, v: contiguous bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 128, 256}; kv_len:
-int32 CUDA tensor [B] of valid key counts (keys at or beyond kv_len[b] never take part).
+q, k, v: bf16 CUDA tensors [B, H, T, D] with D in {32, 64, 128, 256} and d contiguous (the
+single-pass, split and combine calls take other strides as given, so [B, T, H, D] views
+and slices of a packed QKV run without copies; the fused-split and multi-range calls want
+contiguous tensors); kv_len: int32 CUDA tensor [B] of valid key counts (keys at or beyond
+kv_len[b] never take part).
 The computation runs in the hand-written kernels of the C library built from csrc/;
 this package only marshals arguments.
 """
