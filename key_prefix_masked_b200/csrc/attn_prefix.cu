@@ -217,22 +217,30 @@ __device__ __forceinline__ void combine_row(const float* __restrict__ part_out, 
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         L = M + logf(s);
-        for (int c = 0; c < C; ++c) {
-            const float w = expf(ld_part<float, FRESH>(part_lse + c * rows + row) - L);
-            if (w == 0.0f) continue;   // an empty chunk (lse_c = -inf) adds nothing
-            const float* src = part_out + (static_cast<long long>(c) * rows + row) * D + lane * PER;
-            if constexpr (PER % 4 == 0) {
+        // Chunk weights 32 at a time, one per lane, broadcast by shuffle: the partial loads
+        // of consecutive chunks then depend on nothing loaded in the loop and overlap.  An
+        // empty chunk (lse_c = -inf, partial stored as zeros) has weight 0 and adds 0.
+        for (int cb = 0; cb < C; cb += 32) {
+            const int c_l = cb + lane;
+            const float w_l = c_l < C ? expf(ld_part<float, FRESH>(part_lse + c_l * rows + row) - L) : 0.0f;
+            const int nc = min(32, C - cb);
+#pragma unroll 4
+            for (int t = 0; t < nc; ++t) {
+                const float w = __shfl_sync(0xffffffffu, w_l, t);
+                const float* src = part_out + (static_cast<long long>(cb + t) * rows + row) * D + lane * PER;
+                if constexpr (PER % 4 == 0) {
 #pragma unroll
-                for (int e = 0; e < PER; e += 4) {
-                    const float4 v4 = ld_part<float4, FRESH>(reinterpret_cast<const float4*>(src + e));
-                    acc[e] += w * v4.x;
-                    acc[e + 1] += w * v4.y;
-                    acc[e + 2] += w * v4.z;
-                    acc[e + 3] += w * v4.w;
+                    for (int e = 0; e < PER; e += 4) {
+                        const float4 v4 = ld_part<float4, FRESH>(reinterpret_cast<const float4*>(src + e));
+                        acc[e] += w * v4.x;
+                        acc[e + 1] += w * v4.y;
+                        acc[e + 2] += w * v4.z;
+                        acc[e + 3] += w * v4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < PER; ++e) acc[e] += w * ld_part<float, FRESH>(src + e);
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] += w * ld_part<float, FRESH>(src + e);
             }
         }
     }
