@@ -176,9 +176,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             tma_prefetch_map(&tm_v);
             if (leader) mbar_arrive_expect_tx(PBAR(PB_Q), 2 * C::Q_BYTES);
             const uint32_t lq = mapa_shared(PBAR(PB_Q), 0);
+            // Q is read once: evict it first.  Every pair of the head streams the head's K/V:
+            // keep those lines in L2 ahead of Q and of the output stream.
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
 #pragma unroll
             for (int blk = 0; blk < C::NBLK; ++blk)
-                tma_load_4d_pair(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, h, b, lq);
+                tma_load_4d_pair_hint(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, h, b, lq, pol_q);
             int slot = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -195,13 +199,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
 #pragma unroll
                     for (int c = 0; c < C::NBLK; ++c)
                         if (!(drop && c == 0))
-                            tma_load_4d_pair(dst + c * C::KBLK_BYTES, &tm_k, c * 64, key0 + static_cast<int>(rank) * C::KH,
-                                             h, b, lfull);
+                            tma_load_4d_pair_hint(dst + c * C::KBLK_BYTES, &tm_k, c * 64,
+                                                  key0 + static_cast<int>(rank) * C::KH, h, b, lfull, pol_kv);
                 } else {
 #pragma unroll
                     for (int c = 0; c < C::NBLK / 2; ++c)
-                        tma_load_4d_pair(dst + c * C::VBLK_BYTES, &tm_v, static_cast<int>(rank) * (D / 2) + c * 64,
-                                         key0, h, b, lfull);
+                        tma_load_4d_pair_hint(dst + c * C::VBLK_BYTES, &tm_v, static_cast<int>(rank) * (D / 2) + c * 64,
+                                              key0, h, b, lfull, pol_kv);
                 }
                 if (++slot == C::NSLOTS) {
                     slot = 0;
@@ -547,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     v4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
                     v4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
                     v4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-                    *reinterpret_cast<uint4*>(dst + e) = v4;
+                    __stcs(reinterpret_cast<uint4*>(dst + e), v4);   // streaming: out is not read again
                 }
             }
         }

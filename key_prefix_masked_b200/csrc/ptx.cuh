@@ -202,6 +202,26 @@ __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* map, 
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster)
         : "memory");
 }
+// The same copy with an L2 eviction-priority policy (from l2_policy_*) for the bytes it reads.
+__device__ __forceinline__ void tma_load_4d_pair_hint(uint32_t dst, const void* map, int x, int y, int z, int w,
+                                                      uint32_t bar_cluster, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster), "l"(policy)
+        : "memory");
+}
+// L2 policies: lines read under evict_last stay in L2 ahead of normal and evict_first lines.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
 // Pair MMAs (M = 256: 128 rows in each CTA's TMEM; B split along N between the CTAs).
 __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
