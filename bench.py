@@ -482,14 +482,23 @@ def _oracle_sample(w, case, n_rows, seed=0):
     return rows, dt, flops
 
 
+def _rows_for(w, case, seconds: float) -> int:
+    """Number of query rows whose oracle sample takes about `seconds` on the host cores.
+    Small samples run below the cores' parallel efficiency, so the estimate is grown
+    geometrically before it is scaled."""
+    _oracle_sample(w, case, 1, seed=7)          # first call: thread pool start-up, page faults
+    n = 4
+    _, dt, _ = _oracle_sample(w, case, n, seed=8)
+    while dt < 0.25 * seconds and n < w.Tq:
+        n = min(w.Tq, n * 4)
+        _, dt, _ = _oracle_sample(w, case, n, seed=9)
+    return max(1, min(w.Tq, int(n * seconds / max(dt, 1e-4))))
+
+
 def cpu_baseline(w, case, target_s: float):
     import oracle
     cores = oracle.num_threads()
-    _oracle_sample(w, case, 1, seed=7)          # first call: thread pool start-up, page faults
-    rows, dt, flops = _oracle_sample(w, case, 4)
-    if dt < target_s * 0.5:
-        n = max(4, min(w.Tq, int(4 * target_s / max(dt, 1e-3))))
-        rows, dt, flops = _oracle_sample(w, case, n, seed=1)
+    rows, dt, flops = _oracle_sample(w, case, _rows_for(w, case, target_s), seed=1)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{len(rows)} random query rows x {w.H} heads of the {w.name} workload "
@@ -505,9 +514,7 @@ def run_reference(args, rank, world):
     w = synth.WORKLOADS[args.workload]
     case = synth.make_inputs(w, device="cpu", seed=args.seed)
     cores = oracle.num_threads()
-    _oracle_sample(w, case, 1, seed=7)          # first call: thread pool start-up, page faults
-    rows, dt, _ = _oracle_sample(w, case, 4)
-    per_step_rows = max(1, int(args.cpu_seconds / max(args.steps + args.warmup, 1) / max(dt / 4, 1e-4)))
+    per_step_rows = _rows_for(w, case, args.cpu_seconds / max(args.steps + args.warmup, 1))
     for i in range(args.warmup):
         _oracle_sample(w, case, per_step_rows, seed=100 + i)
     times, flops_total = [], 0.0
