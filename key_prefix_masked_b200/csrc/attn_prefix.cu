@@ -53,6 +53,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "attn_prefix.h"
@@ -455,13 +456,15 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         }
         __syncwarp();
     } else if (warp == C::WARP_MMA) {
-        // ================================================================ MMA issuer (one thread)
+        // ================================================================ MMA issuer (one warp)
         // Two readiness events per tile, published by the relay warp: "P_j stored and
         // V_j landed" and "K_{j+2} landed".  Between them the 8 PV and 16 S MMAs of a
         // tile are issued as straight-line code from precomputed descriptors, so the
         // tensor pipe's queue stays fed (the tile's MMA mix alone runs at the tensor
-        // peak; the issuing thread's overhead is what decides the rate).
-        if (lane == 0 && n_tiles > 0) {
+        // peak; the issuing code's overhead is what decides the rate).  The whole warp
+        // runs it converged and its elected lane issues, so the descriptors stay
+        // warp-uniform; every wait decision is lane 0's, broadcast.
+        if (n_tiles > 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(BM, BN, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(BM, D, true);
             constexpr int KG = C::KCH / C::GRP;
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::V_ROWS * C::SW, 8 * C::SW, C::LAYOUT);
             int gi = 0;   // ring group of the next K/V group to consume
             uint32_t consumed = 0;
-            bool ok = wait_bar(BAR(BAR_Q), 0, abort_flag, wlim);
+            bool ok = __all_sync(0xffffffffu, wait_bar(BAR(BAR_Q), 0, abort_flag, wlim));
             auto ring = [&](int g) { return (gi + g < C::NG) ? gi + g : gi + g - C::NG; };
             auto advance = [&](int n) { gi = (gi + n < C::NG) ? gi + n : gi + n - C::NG; };
             // The relay warp performs the blocking mbarrier waits in this thread's order
@@ -481,17 +484,26 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             // shared-memory load instead of an mbarrier round trip.
             auto next_event = [&]() -> bool {
                 ++consumed;
-                if (ld_acquire_smem(ready_addr) >= consumed) return true;
-                const uint64_t t0 = global_timer_ns();
-                while (true) {
-                    if (ld_acquire_smem(ready_addr) >= consumed) return true;
-                    if (*abort_flag) return false;
-                    if (global_timer_ns() - t0 > wlim) {
-                        *abort_flag = 1;
-                        atomicOr(&g_attn_status, STATUS_TIMEOUT);
-                        return false;
+                bool ok_ev = true;
+                if (ld_acquire_smem(ready_addr) < consumed) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (true) {
+                        if (ld_acquire_smem(ready_addr) >= consumed) break;
+                        if (*abort_flag) {
+                            ok_ev = false;
+                            break;
+                        }
+                        if (global_timer_ns() - t0 > wlim) {
+                            if (lane == 0) {
+                                *abort_flag = 1;
+                                atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                            }
+                            ok_ev = false;
+                            break;
+                        }
                     }
                 }
+                return __shfl_sync(0xffffffffu, ok_ev ? 1 : 0, 0) != 0;
             };
             auto issue_s = [&](int j) {
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
@@ -503,14 +515,14 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         const int c = g * C::GRP + cc;
 #pragma unroll
                         for (int kk = 0; kk < C::BLK / 16; ++kk)
-                            mma_ss(d_tmem, q_desc0 + static_cast<uint64_t>(((c * BM * C::SW) >> 4) + kk * 2),
+                            mma_ss_elect(d_tmem, q_desc0 + static_cast<uint64_t>(((c * BM * C::SW) >> 4) + kk * 2),
                                    kd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + kk * 2), IDESC_S,
                                    (c | kk) != 0 ? 1u : 0u);
                     }
                 }
 #pragma unroll
-                for (int g = 0; g < KG; ++g) tc_commit(BAR(BAR_EMPTY + ring(g)));
-                tc_commit(BAR(BAR_S + (j & 1)));
+                for (int g = 0; g < KG; ++g) tc_commit_elect(BAR(BAR_EMPTY + ring(g)));
+                tc_commit_elect(BAR(BAR_S + (j & 1)));
                 advance(KG);
             };
             auto issue_pv = [&](int j) {
@@ -530,18 +542,18 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 #pragma unroll
                         for (int kk = 0; kk < C::V_ROWS / 16; ++kk) {
                             const int kb = (g * C::GRP + cc) * (C::V_ROWS / 16) + kk;
-                            mma_ts(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                            mma_ts_elect(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
                                    vd + static_cast<uint64_t>(((cc * C::SLOT) >> 4) + ((kk * 16 * C::SW) >> 4)),
                                    IDESC_PV, kb == 0 ? acc0 : 1u);
                         }
                     }
                 }
 #pragma unroll
-                for (int g = 0; g < VG; ++g) tc_commit(BAR(BAR_EMPTY + ring(g)));
+                for (int g = 0; g < VG; ++g) tc_commit_elect(BAR(BAR_EMPTY + ring(g)));
                 // One phase per PV on the accumulator's barrier: the softmax group waits
                 // it before rescaling O or reusing the P buffer, the epilogue before reading.
-                tc_commit(BAR(BAR_PVD + (C::DUAL ? (j & 1) : 0)));
-                if (j == n_tiles - 1) tc_commit(BAR(BAR_OFIN));
+                tc_commit_elect(BAR(BAR_PVD + (C::DUAL ? (j & 1) : 0)));
+                if (j == n_tiles - 1) tc_commit_elect(BAR(BAR_OFIN));
                 advance(VG);
             };
             if (ok) ok = next_event();
@@ -595,7 +607,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 }
             }
             // Drain: every MMA issued completes before TMEM is released.
-            tc_commit(BAR(BAR_DRAIN));
+            tc_commit_elect(BAR(BAR_DRAIN));
+            __syncwarp();
             wait_bar_drain(BAR(BAR_DRAIN), 0, wlim);
         }
         __syncwarp();
@@ -917,8 +930,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-unsigned long long g_wait_ns = 1000000000ull;
-unsigned g_debug = 0;
+// Test hooks (attn_set_wait_limit_ns, attn_set_debug_flags): process-wide settings read
+// by every launch that starts after they are written, from any host thread.
+std::atomic<unsigned long long> g_wait_ns{1000000000ull};
+std::atomic<unsigned> g_debug{0u};
 
 EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
@@ -968,29 +983,29 @@ attn_status check_args(const void* q, const void* k, const void* v, const void* 
     return ATTN_OK;
 }
 
-// Device must be compute capability 10.0 (B200 / sm_100a).  Cached per device ordinal.
+// Device must be compute capability 10.0 (B200 / sm_100a).  Cached per device ordinal
+// (0 = not looked up yet, 1 = supported, 2 = not supported); host threads may race on an
+// entry, and every one of them writes the same value.
 attn_status check_device() {
-    static int cached[64];
-    static std::once_flag once;
-    std::call_once(once, [] {
-        for (int i = 0; i < 64; ++i) cached[i] = -1;
-    });
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
     if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
-    if (cached[dev] < 0) {
+    int c = cached[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_CUDA;
         }
-        cached[dev] = (major == 10 && minor == 0) ? 1 : 0;
+        c = (major == 10 && minor == 0) ? 1 : 2;
+        cached[dev].store(c, std::memory_order_relaxed);
     }
-    return cached[dev] ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+    return c == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
 // A [B, H, T, D] bf16 tensor at element strides s (d contiguous) as a 4-D TMA map with
@@ -1094,8 +1109,8 @@ Params base_params(const int32_t* kv_len, int B, int H, int Tq, int Tk, int D, f
     prm.out_sb = so.b;
     prm.out_sh = so.h;
     prm.out_st = so.t;
-    prm.wait_ns = g_wait_ns;
-    prm.debug = g_debug;
+    prm.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    prm.debug = g_debug.load(std::memory_order_relaxed);
     return prm;
 }
 
@@ -1297,9 +1312,11 @@ attn_status attn_get_device_status(cudaStream_t stream) {
     return ATTN_OK;
 }
 
-void attn_set_wait_limit_ns(uint64_t ns) { g_wait_ns = ns < 1000000ull ? 1000000ull : ns; }
+void attn_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns.store(ns < 1000000ull ? 1000000ull : ns, std::memory_order_relaxed);
+}
 
-void attn_set_debug_flags(unsigned flags) { g_debug = flags; }
+void attn_set_debug_flags(unsigned flags) { g_debug.store(flags, std::memory_order_relaxed); }
 
 const char* attn_status_string(attn_status s) {
     switch (s) {
@@ -1325,24 +1342,58 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SC
 
 namespace {
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// The driver's id of the current context (0 if it cannot be read).  A device reset or a
+// context torn down and created again gets a new id, and may load the module -- and so
+// the scratch array -- at a new address.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[64] = {};
+unsigned long long g_noalloc_ctx[64] = {};
 
-// Device address of the scratch array on the current device (nullptr on failure).
+// Device address of the scratch array on the current device (nullptr on failure).  It is
+// looked up with cudaGetSymbolAddress the first time a device is used, and again whenever
+// that device's current context has changed since (a reset between calls).
 void* noalloc_scratch_on_current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return nullptr;
     }
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
         g_noalloc_ptr[dev] = ptr;
+        // read after the lookup, which creates the primary context if none existed yet
+        g_noalloc_ctx[dev] = current_context_id();
     }
     return g_noalloc_ptr[dev];
 }

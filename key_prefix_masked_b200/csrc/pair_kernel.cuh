@@ -272,7 +272,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
         __syncwarp();
     } else if (warp == C::WARP_MMA) {
         // ================================================================ MMA issuer (leader)
-        if (leader && lane == 0 && n_tiles > 0) {
+        // The whole warp runs the issuing code converged and its elected lane issues every
+        // MMA and commit, so the descriptors stay warp-uniform (measured on B200: 68 cycles
+        // per MMA issued this way against 83 from one thread of a divergent branch; at
+        // D=256 an S MMA executes in 64, so the issue rate bounds the S phase).  Every wait
+        // decision is lane 0's, broadcast, so the warp stays converged.
+        if (leader && n_tiles > 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(2 * C::ROWS, BN, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(2 * C::ROWS, D, true);
             const uint64_t q_desc0 = make_smem_desc(sQ_addr, 16, 1024, 2);
@@ -280,18 +285,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             const uint64_t v_desc0 = make_smem_desc(sKV_addr, C::VBLK_BYTES, 1024, 2);
             int slot = 0;
             uint32_t consumed = 0;
+            auto uniform = [&](bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; };
             auto poll_ge = [&](uint32_t addr, uint32_t need) -> bool {
-                if (ld_acquire_cluster_smem(addr) >= need) return true;
-                const uint64_t t0 = global_timer_ns();
-                while (true) {
-                    if (ld_acquire_cluster_smem(addr) >= need) return true;
-                    if (*abort_flag) return false;
-                    if (global_timer_ns() - t0 > wlim) {
-                        *abort_flag = 1;
-                        atomicOr(&g_attn_status, STATUS_TIMEOUT);
-                        return false;
+                bool ok_p = true;
+                if (ld_acquire_cluster_smem(addr) < need) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (true) {
+                        if (ld_acquire_cluster_smem(addr) >= need) break;
+                        if (*abort_flag) {
+                            ok_p = false;
+                            break;
+                        }
+                        if (global_timer_ns() - t0 > wlim) {
+                            if (lane == 0) {
+                                *abort_flag = 1;
+                                atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                            }
+                            ok_p = false;
+                            break;
+                        }
                     }
                 }
+                return uniform(ok_p);
             };
             auto slot_desc = [&](uint64_t d0) { return d0 + static_cast<uint64_t>(slot) * (C::SLOT >> 4); };
             auto next_slot = [&]() { slot = (slot + 1 == C::NSLOTS) ? 0 : slot + 1; };
@@ -305,11 +320,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
 #pragma unroll
                 for (int t = 0; t < D / 16; ++t) {
                     const int c = t >> 2, kk = t & 3;
-                    mma_ss_pair(d_tmem, q_desc0 + static_cast<uint64_t>(((c * C::ROWS * 128) >> 4) + kk * 2),
-                                kd + static_cast<uint64_t>(((c * C::KBLK_BYTES) >> 4) + kk * 2), IDESC_S, t != 0);
+                    mma_ss_pair_elect(d_tmem, q_desc0 + static_cast<uint64_t>(((c * C::ROWS * 128) >> 4) + kk * 2),
+                                      kd + static_cast<uint64_t>(((c * C::KBLK_BYTES) >> 4) + kk * 2), IDESC_S, t != 0);
                 }
-                tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
-                tc_commit_pair(PBAR(PB_S + (j & 1)), 0x3);
+                tc_commit_pair_elect(PBAR(PB_EMPTY + slot), 0x3);
+                tc_commit_pair_elect(PBAR(PB_S + (j & 1)), 0x3);
                 next_slot();
             };
             auto issue_pv = [&](int j) {
@@ -319,16 +334,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     // P_j stored in both CTAs: probed here, without suspending
                     const uint32_t pb = PBAR(PB_P + (j & 1));
                     const uint32_t par = (j >> 1) & 1;
-                    if (!mbar_test_wait(pb, par)) {
+                    if (!uniform(mbar_test_wait(pb, par))) {
                         const uint64_t t0 = global_timer_ns();
-                        while (!mbar_test_wait(pb, par)) {
-                            if (*abort_flag) {
+                        while (true) {
+                            if (uniform(mbar_test_wait(pb, par))) break;
+                            if (uniform(*abort_flag != 0)) {
                                 ok = false;
                                 return;
                             }
-                            if (global_timer_ns() - t0 > wlim) {
-                                *abort_flag = 1;
-                                atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                            if (uniform(global_timer_ns() - t0 > wlim)) {
+                                if (lane == 0) {
+                                    *abort_flag = 1;
+                                    atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                                }
                                 ok = false;
                                 return;
                             }
@@ -344,13 +362,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 const uint64_t vd = slot_desc(v_desc0);
 #pragma unroll
                 for (int kb = 0; kb < BN / 16; ++kb)
-                    mma_ts_pair(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV, kb == 0 ? acc0 : 1u);
-                tc_commit_pair(PBAR(PB_EMPTY + slot), 0x3);
+                    mma_ts_pair_elect(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
+                                      vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV, kb == 0 ? acc0 : 1u);
+                tc_commit_pair_elect(PBAR(PB_EMPTY + slot), 0x3);
                 // Each O barrier completes exactly once, so a parity-0 wait on it cannot
                 // be confused by a later phase.
-                if (!C::DUAL && j == n_tiles - 2) tc_commit_pair(PBAR(PB_OPREV), 0x3);
-                if (j == n_tiles - 1) tc_commit_pair(PBAR(PB_OLAST), 0x3);
+                if (!C::DUAL && j == n_tiles - 2) tc_commit_pair_elect(PBAR(PB_OPREV), 0x3);
+                if (j == n_tiles - 1) tc_commit_pair_elect(PBAR(PB_OLAST), 0x3);
                 next_slot();
             };
             if (ok) issue_s(0);
@@ -360,7 +378,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 issue_pv(j);
                 if (ok && j + 2 < n_tiles) issue_s(j + 2);
             }
-            tc_commit_pair(PBAR(PB_DRAIN), 0x1);
+            tc_commit_pair_elect(PBAR(PB_DRAIN), 0x1);
+            __syncwarp();
             wait_bar_drain(PBAR(PB_DRAIN), 0, wlim);
         }
         __syncwarp();

@@ -29,7 +29,7 @@
  *   - "Broadcast SDPA attn_mask instead of materializing a per-head copy", section
  *     "What": one mask per batch element serves every head.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent (each one applied the same way by every mode):
  *   - lse is the natural logarithm of sum_j exp(scale * q.k_j), scale included;
  *   - n = 0 gives out = 0 and lse = -inf (the pages leave an empty prefix undefined);
  *   - key selection is exact: keys j >= n are never read in truncation mode.
@@ -273,7 +273,7 @@ int oracle_lse_combine(const double* part_out, const double* part_lse, int C, lo
  * gathered-shards case of "Add sequence-parallel multi-GPU inference ...", section
  * "Sequence-parallel inference": each device's context K/V is gathered with padded key
  * slots, so the valid keys are one range per shard rather than one prefix.
- * Readings where the pages are silent (listed in the design doc):
+ * Readings where the pages are silent:
  *   - a segment is intersected with [0, Tk); a negative length counts as 0;
  *   - a key that lies in two segments takes part twice (the segments are concatenated);
  *   - the concatenation is cut after Tk keys;

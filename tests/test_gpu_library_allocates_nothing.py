@@ -3,7 +3,7 @@
 After one warm-up call per entry point (which may load the kernels' code onto the
 device), further calls through the C ABI with caller-owned buffers must leave the
 device's free memory exactly where it was, at every head dim and for the single-pass,
-split + combine, fused-split and multi-range entries.
+split + combine, fused-split, multi-range and no-allocation split-KV entries.
 """
 import ctypes
 
@@ -60,6 +60,10 @@ def test_entry_points_allocate_nothing(lib, D):
                                             P(seg_start.data_ptr()), P(seg_len.data_ptr()), 2, P(seg_ws.data_ptr()),
                                             P(out.data_ptr()), P(lse.data_ptr()), B, H, Tq, Tk, D, scale,
                                             stream) == 0
+        assert lib.attn_split_workspace_bytes(C, B, H, Tq, D) <= 64 * 1024 * 1024
+        assert lib.attn_prefix_fwd_splitkv_noalloc(P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()),
+                                                   P(kv.data_ptr()), C, P(out.data_ptr()), P(lse.data_ptr()),
+                                                   B, H, Tq, Tk, D, scale, stream) == 0
 
     calls()                      # warm-up: module and kernel loading
     before = _free_bytes()

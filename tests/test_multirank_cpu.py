@@ -1,5 +1,5 @@
 """The multi-rank plumbing of bench.py on CPU: two gloo ranks on 127.0.0.1 agree on the
-max-over-ranks step time and the whole-job throughput counts every rank's work."""
+max-over-ranks step time, and replicas count every rank's work in the whole-job flops."""
 import os
 import socket
 import subprocess
@@ -17,8 +17,13 @@ rank, world, _ = bench.dist_setup(2)
 ms = 10.0 + 5.0 * rank                      # rank 1 is the slow one
 bench.barrier(world)
 slowest = bench.max_over_ranks(ms, world)
-value = bench.whole_job_tflops(1e12, world, slowest)
-print(json.dumps({"rank": rank, "world": world, "slowest": slowest, "value": value}), flush=True)
+import types, torch, synth
+w = synth.Workload("rep", 1, 1, 32, 5, 40, (40,), 1.0, False)
+prob = bench.Problem(None, w, types.SimpleNamespace(seed=0, split_mode="separate"), rank, world, "replicas",
+                     torch.device("cpu"))
+value = prob.flops_job / (slowest * 1e-3) / 1e12
+print(json.dumps({"rank": rank, "world": world, "slowest": slowest, "value": value,
+                  "flops_total": prob.flops_total}), flush=True)
 import torch.distributed as dist
 dist.destroy_process_group()
 '''
@@ -50,13 +55,8 @@ def test_two_gloo_ranks_take_the_max_and_count_all_work(tmp_path):
         outs.append(json.loads(out.strip().splitlines()[-1]))
     for o in outs:
         assert o["world"] == 2 and o["slowest"] == 15.0
-        assert abs(o["value"] - 2 * 1e12 / 15e-3 / 1e12) < 1e-9
-
-
-def test_whole_job_tflops_single_rank():
-    sys.path.insert(0, ROOT)
-    import bench
-    assert abs(bench.whole_job_tflops(9.0112e13, 1, 66.7) - 1351.0) < 1.0
+        assert o["flops_total"] == 4.0 * 1 * 5 * 40 * 32
+        assert abs(o["value"] - 2 * o["flops_total"] / 15e-3 / 1e12) < 1e-12
 
 
 def test_reference_arm_runs_on_host_cores():

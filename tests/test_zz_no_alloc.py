@@ -4,15 +4,19 @@ It serves callers that cannot call cudaMalloc themselves -- code that only recei
 inputs and outputs from a framework allocator or a fixed memory plan.  Its partials live
 in the library's own device array, so the test checks, through the C ABI, that two calls
 in a row (the second reusing whatever the first left in that array) give what the
-existing allocate-your-own-workspace split-KV path gives, within the parity tolerance.
+existing allocate-your-own-workspace split-KV path gives, and what the fp64 oracle
+gives, within the parity tolerance.  Empty and one-key prefixes are among the rows.
 
-This file is collected last on purpose.
+The file name sorts after every other test file, so a run that stops at its first
+failure has run all the other tests before this one.  Nothing here depends on that
+order: the test passes alone in a fresh process and after the others.
 """
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 import synth
 from parity import assert_lse_close, assert_out_close
 
@@ -52,9 +56,11 @@ def test_oversized_workspace_is_rejected_before_any_cuda_call(lib):
 def test_noalloc_matches_split_kv_path_on_two_calls(lib):
     import key_prefix_masked_b200 as kp
     cases = [
-        # first call: larger footprint; the second is smaller and reuses the array
+        # first call: larger footprint; the next ones are smaller and reuse the array
         (synth.random_case(2, 4, 300, 3000, 256, (3000, 1111), seed=31, std=0.5), 6),
         (synth.random_case(3, 2, 130, 900, 64, (0, 1, 899), seed=32), 3),
+        (synth.random_case(2, 3, 77, 500, 128, (129, 0), seed=33), 4),
+        (synth.random_case(2, 2, 64, 96, 32, (40, 1), seed=34), 2),
     ]
     for case, C in cases:
         g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in case.items()}
@@ -67,5 +73,8 @@ def test_noalloc_matches_split_kv_path_on_two_calls(lib):
                                                       g["scale"])
         torch.cuda.synchronize()
         assert kp.device_status() == kp.ATTN_OK
-        assert_out_close(out, ref_out.double().cpu().numpy(), what="noalloc out")
-        assert_lse_close(lse, ref_lse.double().cpu().numpy(), what="noalloc lse")
+        assert_out_close(out, ref_out.double().cpu().numpy(), what="noalloc out vs split path")
+        assert_lse_close(lse, ref_lse.double().cpu().numpy(), what="noalloc lse vs split path")
+        o_out, o_lse = oracle.attn_prefix(case["q"], case["k"], case["v"], case["kv_len_list"], case["scale"])
+        assert_out_close(out, o_out, what="noalloc out vs oracle")
+        assert_lse_close(lse, o_lse, what="noalloc lse vs oracle")
