@@ -196,7 +196,8 @@ attn_status attn_prefix_fwd_segments(const void* q, const void* k, const void* v
  *   exceeds ATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_INVALID_ARG before any
  *   CUDA call.
  *   The first call on a device looks up the array's device address (with that device
- *   current); make that first call before any stream capture.
+ *   current); make that first call before any stream capture.  After a device reset
+ *   (a new context on the device) the next call looks the address up again.
  *   Every call shares the one array and leaves its partials there; each call writes
  *   every partial it reads, so nothing needs clearing, but calls whose work overlaps on
  *   the GPU (other streams, other host threads) race on the array and must be serialised
@@ -218,7 +219,9 @@ attn_status attn_get_device_status(cudaStream_t stream);
  * exit, and raises ATTN_ERR_TIMEOUT.  Values below 1e6 are raised to 1e6. */
 void attn_set_wait_limit_ns(uint64_t ns);
 
-/* Test hook.  ATTN_DEBUG_DROP_COPY makes the copy producer of the next launches
+/* Test hooks, for tests only.  They are process-wide settings (atomics) that apply to
+ * every launch, from any host thread, started after the call.
+ * ATTN_DEBUG_DROP_COPY makes the copy producer of the next launches
  * announce one key-tile copy without issuing it, so that the consumer's bounded wait
  * runs out (exercises the ATTN_ERR_TIMEOUT path without faulting anything).  0 = off. */
 #define ATTN_DEBUG_DROP_COPY 1u

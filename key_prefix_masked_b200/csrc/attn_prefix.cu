@@ -482,13 +482,19 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             // The relay warp performs the blocking mbarrier waits in this thread's order
             // and publishes how many events have completed; polling that word costs a
             // shared-memory load instead of an mbarrier round trip.
+            // lane 0 reads the relay's count and broadcasts it (one shared-memory load per poll)
+            auto poll_word = [&](uint32_t addr) -> uint32_t {
+                uint32_t v = 0;
+                if (lane == 0) v = ld_acquire_smem(addr);
+                return __shfl_sync(0xffffffffu, v, 0);
+            };
             auto next_event = [&]() -> bool {
                 ++consumed;
                 bool ok_ev = true;
-                if (ld_acquire_smem(ready_addr) < consumed) {
+                if (poll_word(ready_addr) < consumed) {
                     const uint64_t t0 = global_timer_ns();
                     while (true) {
-                        if (ld_acquire_smem(ready_addr) >= consumed) break;
+                        if (poll_word(ready_addr) >= consumed) break;
                         if (*abort_flag) {
                             ok_ev = false;
                             break;

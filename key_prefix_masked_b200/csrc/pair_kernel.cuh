@@ -286,12 +286,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             int slot = 0;
             uint32_t consumed = 0;
             auto uniform = [&](bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; };
+            // lane 0 reads the relay's count and broadcasts it (one shared-memory load per poll)
+            auto poll_word = [&](uint32_t addr) -> uint32_t {
+                uint32_t v = 0;
+                if (lane == 0) v = ld_acquire_cluster_smem(addr);
+                return __shfl_sync(0xffffffffu, v, 0);
+            };
             auto poll_ge = [&](uint32_t addr, uint32_t need) -> bool {
                 bool ok_p = true;
-                if (ld_acquire_cluster_smem(addr) < need) {
+                if (poll_word(addr) < need) {
                     const uint64_t t0 = global_timer_ns();
                     while (true) {
-                        if (ld_acquire_cluster_smem(addr) >= need) break;
+                        if (poll_word(addr) >= need) break;
                         if (*abort_flag) {
                             ok_p = false;
                             break;
