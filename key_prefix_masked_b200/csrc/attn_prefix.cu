@@ -55,6 +55,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "attn_prefix.h"
 #include "ptx.cuh"
@@ -494,6 +495,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 if (poll_word(ready_addr) < consumed) {
                     const uint64_t t0 = global_timer_ns();
                     while (true) {
+                        __nanosleep(32);   // a spinning poll takes issue slots from the softmax warps beside it
                         if (poll_word(ready_addr) >= consumed) break;
                         if (*abort_flag) {
                             ok_ev = false;
@@ -1070,7 +1072,9 @@ attn_status launch_fwd_pair(const void* q, const void* k, const void* v, const S
     prm.n_qtiles = (prm.Tq + 2 * C::ROWS - 1) / (2 * C::ROWS);
     const long long grid = 2LL * prm.n_qtiles * BH * (SPLIT ? prm.num_splits : 1);
     if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    auto kern = attn::attn_fwd_pair_kernel<D, SPLIT>;
+    // the pipelined softmax (D=128) is specialised on the sign of the scale
+    auto kern = (C::PIPE && !(prm.scale_log2 > 0.0f)) ? attn::attn_fwd_pair_kernel<D, SPLIT, false>
+                                                      : attn::attn_fwd_pair_kernel<D, SPLIT, true>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
