@@ -30,8 +30,8 @@
 // barrier (the remote mbarrier arrive with default semantics -- release at CTA scope --
 // which is the cross-CTA handshake the pair pipelines are built on; a cluster-scope
 // release costs ~450-1100 cycles and made this handshake the critical path).  The relay
-// folds "P_j stored in both CTAs" and "V_j landed" into one event for the MMA warp (at
-// D=128 the MMA warp waits for "P_j stored" itself).
+// publishes "V_j landed" and the K arrivals; the MMA warp waits for "P_j stored in both
+// CTAs" itself.
 //
 // The last, partial key tile of a range is read as the window [k_end - 128, k_end):
 // every row copied is a valid key (or a zero-filled row at a negative coordinate), and
@@ -63,10 +63,11 @@ struct PairCfg {
     static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
     static constexpr int NSLOTS = NSLOTS_FIT < PAIR_MAX_SLOTS ? NSLOTS_FIT : PAIR_MAX_SLOTS;
     static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
-    // Who waits for "P_j stored": at D=128 the MMA warp waits on the P barrier itself,
-    // which takes the relay's wake-up off the P -> PV handshake; at D=256 the MMA warp has twice the MMAs to issue per tile and the
-    // relay keeps that wait (measured: +2 to +4 % at D=128, -1.5 % at D=256 the other way).
-    static constexpr bool MMA_WAITS_P = D <= 128;
+    // Who waits for "P_j stored": the MMA warp itself, with a suspending try_wait, which
+    // takes the relay's wake-up off the P -> PV handshake (measured, same-box A/B against
+    // the relay doing that wait: +6.5 % on icl and +6.1 % on ragged at D=256, +2 to +4 %
+    // at D=128; a spinning test_wait from one thread had cost 1.5 % at D=256).
+    static constexpr bool MMA_WAITS_P = true;
     static_assert(D == 128 || D == 256, "pair head dims");
     static_assert(NSLOTS >= 4, "pair ring depth");
     static_assert(SMEM_BYTES <= SMEM_LIMIT && 2 * SMEM_BYTES > SMEM_LIMIT, "one CTA per SM, within budget");
