@@ -58,7 +58,6 @@
 
 #include <atomic>
 #include <mutex>
-#include <type_traits>
 
 #include "attn_prefix.h"
 #include "ptx.cuh"
@@ -1061,9 +1060,7 @@ attn_status launch_fwd_pair(const void* q, const void* k, const void* v, const S
     prm.n_qtiles = (prm.Tq + 2 * C::ROWS - 1) / (2 * C::ROWS);
     const long long grid = 2LL * prm.n_qtiles * BH * (SPLIT ? prm.num_splits : 1);
     if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    // the pipelined softmax (D=128) is specialised on the sign of the scale
-    auto kern = (C::PIPE && !(prm.scale_log2 > 0.0f)) ? attn::attn_fwd_pair_kernel<D, SPLIT, false>
-                                                      : attn::attn_fwd_pair_kernel<D, SPLIT, true>;
+    auto kern = attn::attn_fwd_pair_kernel<D, SPLIT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;

@@ -6,32 +6,30 @@
 // value tile -- keys [64r, 64r + 64) of K, value columns [r*D/2, (r+1)*D/2) of V for
 // CTA rank r.  The leader CTA's MMA warp issues M = 256 tcgen05 MMAs that read A from
 // each CTA and B split across both, so each CTA streams half of every K/V tile (64 KB at
-// D=256, 32 KB at D=128) and one instruction covers 256 rows: at D=256 the five 32 KB
-// ring slots hold 2.5 tiles of look-ahead, at D=128 twelve 16 KB slots hold 6.
+// D=256, 32 KB at D=128) and one instruction covers 256 rows: at D=256 the five 32 KB ring slots hold 2.5 tiles of look-ahead, at D=128 twelve
+// 16 KB slots hold 6.  MMA order: S_0, S_1, then PV_j, S_{j+2} per tile j; P_j is stored
+// over S_j, and S_{j+2} overwrites it only after PV_j has read it (one thread's MMAs run
+// in issue order).
 //
-// TMEM holds NS S buffers (S_j in buffer j % NS, P_j stored over S_j as bf16) and the O
-// accumulator after them: NS = 2 at D=256 (S 256 columns + O 256), NS = 3 at D=128
-// (S 384 + O 128).  MMA order: S_0 .. S_{NS-1}, then PV_j, S_{j+NS} per tile j; S_{j+NS}
-// overwrites P_j only after PV_j has read it (one thread's MMAs run in issue order).
-//
-// Roles (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4 copy
-// producer (both CTAs, into their own memory, completing on the leader's barriers);
+// Roles at D=256 (224 threads per CTA): warps 0-3 softmax + epilogue (both CTAs); warp 4
+// copy producer (both CTAs, into their own memory, completing on the leader's barriers);
 // warp 5 TMEM allocation (both) and MMA issue (leader); warp 6 wait relay (leader).
-//
-// Softmax at D=256 (NS = 2): per tile, the S tile is loaded, its row maximum taken, then
-// the exponentials run; the next S is issued only after this tile's P has been used by
-// PV_j, so the chain P_j -> PV_j -> S_{j+2} -> softmax closes over two tiles.  At D=128
-// (NS = 3) the softmax is pipelined: S_{j+1} is complete while tile j runs, so each warp
-// takes the row maximum of tile j + 1 during tile j's exponentials (loads issued half a
-// tile ahead of their use, a tile body without run-time branches that the compiler can
-// interleave), and the exponential stream of a warp is not broken by a maximum phase.
+// At D=128 the kernel runs in two-group mode (352 threads: softmax warps 0-7, then the
+// same three roles): warpgroup w takes the key tiles j = w (mod 2) with its own running
+// max, row sum and TMEM O accumulator O_w (S_0, S_1, O_0, O_1 fill the 512 columns), so
+// one group's softmax overlaps the other's P -> PV -> S round trip; the two warps that
+// share a sub-partition run their exponentials whenever their tiles are ready (turns in
+// tile order cost 5 to 8 % once the MMA warp stopped spinning); the two partial results
+// are merged exactly at the end by the log-sum-exp rule of split-KV ("Sequence-parallel inference"
+// of "Add sequence-parallel multi-GPU inference ... and a cuDNN flash attention option").
+// S_j is issued after PV_{j-2}, the last PV into O_{j&1} before tile j, so "S_j ready"
+// already means that accumulator is quiescent and the group rescales it without waiting.
 //
 // Each softmax warp of either CTA announces P with one arrival on the leader's P
 // barrier (the remote mbarrier arrive with default semantics -- release at CTA scope --
 // which is the cross-CTA handshake the pair pipelines are built on; a cluster-scope
 // release costs ~450-1100 cycles and made this handshake the critical path).  The relay
-// publishes "V_j landed" and the K arrivals; the MMA warp waits for "P_j stored in both
-// CTAs" itself.
+// publishes the copies' arrivals; the MMA warp waits for "P_j stored in both CTAs" itself.
 //
 // The last, partial key tile of a range is read as the window [k_end - 128, k_end):
 // every row copied is a valid key (or a zero-filled row at a negative coordinate), and
@@ -50,19 +48,19 @@ struct PairCfg {
     static constexpr int KBLK_BYTES = KH * 128;      // one 64-column block of them: 8 KB
     static constexpr int VBLK_BYTES = BN * 128;      // one 64-column block of V: 16 KB
     static constexpr int SLOT = NBLK * KBLK_BYTES;   // one CTA's half of a K or V tile
-    // Three S buffers beside O when they fit (D=128): the pipelined softmax.
-    static constexpr bool PIPE = 3 * BN + D <= static_cast<int>(TMEM_COLS);
-    static constexpr int NS = PIPE ? 3 : 2;          // S / P buffers in TMEM
-    static constexpr uint32_t O_COL = NS * BN;       // O accumulator columns [O_COL, O_COL + D)
-    static constexpr int SM_WARPS = 4;               // softmax warps
+    // Two-group mode (head dim 128): two softmax warpgroups on alternate key tiles, each
+    // with its own O accumulator; S_0, S_1, O_0, O_1 fill the 512 TMEM columns.
+    static constexpr bool DUAL = O_COL + 2 * D <= TMEM_COLS;
+    static constexpr int SM_WARPS = DUAL ? 8 : 4;    // softmax warps
     static constexpr int WARP_PROD = SM_WARPS;       // copy producer (both CTAs)
     static constexpr int WARP_MMA = SM_WARPS + 1;    // TMEM owner (both), MMA issuer (leader)
     static constexpr int WARP_RELAY = SM_WARPS + 2;  // wait relay (leader)
     static constexpr int THREADS = 32 * (SM_WARPS + 3);
     static constexpr int CTRL = 1024;
-    static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL) / SLOT;
+    static constexpr int XCH_BYTES = DUAL ? 2 * 2 * ROWS * 4 : 0;   // per-group (max, sum) exchange
+    static constexpr int NSLOTS_FIT = (SMEM_LIMIT - Q_BYTES - CTRL - XCH_BYTES) / SLOT;
     static constexpr int NSLOTS = NSLOTS_FIT < PAIR_MAX_SLOTS ? NSLOTS_FIT : PAIR_MAX_SLOTS;
-    static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL;
+    static constexpr int SMEM_BYTES = Q_BYTES + NSLOTS * SLOT + CTRL + XCH_BYTES;
     // Who waits for "P_j stored": the MMA warp itself, with a suspending try_wait, which
     // takes the relay's wake-up off the P -> PV handshake (measured, same-box A/B against
     // the relay doing that wait: +6.5 % on icl and +6.1 % on ragged at D=256, +2 to +4 %
@@ -79,24 +77,20 @@ enum : int {
     PB_Q = 0,
     PB_FULL = 1,     // [PAIR_MAX_SLOTS] slot filled by both CTAs' copies (leader)
     PB_EMPTY = 13,   // [PAIR_MAX_SLOTS] slot consumed (multicast commit, both CTAs)
-    PB_S = 25,       // [3] S_j ready in buffer j % NS (multicast commit, both CTAs)
-    PB_P = 28,       // [3] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
-    PB_PVD = 31,     // [2] pipelined mode: PV_j complete, on j & 1 (multicast commit, both CTAs)
-    PB_OLAST = 33,   // PV_{n-1} complete (multicast commit, both CTAs; completes once)
-    PB_OPREV = 34,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
-    PB_DRAIN = 35,   // leader only
-    PB_NUM = 36
+    PB_S = 25,       // [2] S_j ready (multicast commit, both CTAs)
+    PB_OLAST = 27,   // PV_{n-1} complete (multicast commit, both CTAs; completes once)
+    PB_DRAIN = 28,   // leader only
+    PB_P = 29,       // [2] P_j stored by both CTAs' softmax warps (leader; 8 warp arrivals)
+    PB_OPREV = 31,   // PV_{n-2} complete (multicast commit, both CTAs; completes once)
+    PB_NUM = 32
 };
 static_assert(PB_EMPTY == PB_FULL + PAIR_MAX_SLOTS && PB_S == PB_EMPTY + PAIR_MAX_SLOTS, "pair barrier map");
 
-// POS: the scale is positive (used by the pipelined softmax, which takes the maximum
-// over scores prepared before the exponentials).
-template <int D, bool SPLIT, bool POS>
+template <int D, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
     using C = PairCfg<D>;
-    constexpr int NS = C::NS;
     extern __shared__ __align__(1024) uint8_t smem[];
     // Swizzled tiles need 1024-byte alignment; both CTAs see the same layout, so both
     // return here together (no cluster barrier has been reached yet).
@@ -149,15 +143,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             mbar_init(PBAR(PB_FULL + s), 1);
             mbar_init(PBAR(PB_EMPTY + s), 1);
         }
-        for (int i = 0; i < 3; ++i) {
-            mbar_init(PBAR(PB_S + i), 1);
-            mbar_init(PBAR(PB_P + i), 8);
-        }
-        mbar_init(PBAR(PB_PVD + 0), 1);
-        mbar_init(PBAR(PB_PVD + 1), 1);
+        mbar_init(PBAR(PB_S + 0), 1);
+        mbar_init(PBAR(PB_S + 1), 1);
         mbar_init(PBAR(PB_OLAST), 1);
         mbar_init(PBAR(PB_OPREV), 1);
         mbar_init(PBAR(PB_DRAIN), 1);
+        mbar_init(PBAR(PB_P + 0), 8);
+        mbar_init(PBAR(PB_P + 1), 8);
         words[1] = 0u;
         words[2] = 0u;
         fence_mbar_init();
@@ -174,7 +166,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
 
     if (warp == C::WARP_PROD) {
         // ================================================================ producer (both CTAs)
-        // Copies in the MMA warp's consumption order: K_0 .. K_{NS-1}, then V_j, K_{j+NS}.
         if (lane == 0 && n_tiles > 0) {
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
@@ -217,11 +208,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     phase ^= 1u;
                 }
             };
-            for (int i = 0; i < NS && i < n_tiles; ++i) item(true, i);
+            item(true, 0);
+            if (n_tiles > 1) item(true, 1);
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
                 item(false, j);
-                if (j + NS < n_tiles) item(true, j + NS);
+                if (j + 2 < n_tiles) item(true, j + 2);
             }
             if (!ok) {
                 // Copies already issued complete on the leader's barriers; give them time to
@@ -234,10 +226,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
         __syncwarp();
     } else if (warp == C::WARP_RELAY) {
         // ================================================================ wait relay (leader)
-        // Waits on Q and, in the MMA warp's consumption order, on K_0 .. K_{NS-1}, then per
-        // tile "V_j landed and P_j stored in both CTAs" (without P_j when the MMA warp
-        // probes it itself) and K_{j+NS}; publishes the count of completed events with a
-        // release store.
+        // Waits on Q and, in the MMA warp's consumption order, on K_0, K_1, then per tile
+        // V_j and K_{j+2}; publishes the count of completed events with a release store.
         if (leader && lane == 0 && n_tiles > 0) {
             uint32_t seq = 0;
             bool ok = wait_bar(PBAR(PB_Q), 0, abort_flag, wlim);
@@ -254,25 +244,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             auto publish = [&]() {
                 if (ok) st_release_smem(seq_addr, ++seq);
             };
-            for (int i = 0; i < NS && i < n_tiles; ++i) {
-                item();  // K_i
+            item();  // K_0
+            publish();
+            if (n_tiles > 1) {
+                item();  // K_1
                 publish();
             }
-            int pb = 0;          // j % NS
-            uint32_t ppar = 0;   // (j / NS) & 1
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
-                item();  // V_j: waited first, as it has usually landed long before P_j, so
-                         // that "P_j stored" reaches the MMA warp one wait sooner
-                if constexpr (!C::MMA_WAITS_P) ok = ok && wait_bar(PBAR(PB_P + pb), ppar, abort_flag, wlim);
+                item();  // V_j
+                if constexpr (!C::MMA_WAITS_P)
+                    ok = ok && wait_bar(PBAR(PB_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
                 publish();
-                if (j + NS < n_tiles) {
-                    item();  // K_{j+NS}
+                if (j + 2 < n_tiles) {
+                    item();  // K_{j+2}
                     publish();
-                }
-                if (++pb == NS) {
-                    pb = 0;
-                    ppar ^= 1u;
                 }
             }
         }
@@ -300,8 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 return __shfl_sync(0xffffffffu, v, 0);
             };
             // A failed poll backs off (nanosleep) before the next one: this warp shares its
-            // sub-partition with softmax warp 1, and a spinning poll takes that warp's issue
-            // slots (stamps: warp 1 then announced P 770 cycles after the other warps).
+            // sub-partition with a softmax warp, and a spinning poll takes its issue slots.
             auto poll_ge = [&](uint32_t addr, uint32_t need) -> bool {
                 bool ok_p = true;
                 if (poll_word(addr) < need) {
@@ -332,8 +317,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 ok = poll_ge(seq_addr, ++consumed);     // K_j halves landed in both CTAs
                 if (!ok) return;
                 tc_fence_after();
-                const int sb = j % NS;
-                const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb) * BN;
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
                 const uint64_t kd = slot_desc(k_desc0);
 #pragma unroll
                 for (int t = 0; t < D / 16; ++t) {
@@ -342,18 +326,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                                       kd + static_cast<uint64_t>(((c * C::KBLK_BYTES) >> 4) + kk * 2), IDESC_S, t != 0);
                 }
                 tc_commit_pair_elect(PBAR(PB_EMPTY + slot), 0x3);
-                tc_commit_pair_elect(PBAR(PB_S + sb), 0x3);
+                tc_commit_pair_elect(PBAR(PB_S + (j & 1)), 0x3);
                 next_slot();
             };
             auto issue_pv = [&](int j) {
-                ok = poll_ge(seq_addr, ++consumed);   // V_j halves landed (and P_j stored, via the relay)
+                ok = poll_ge(seq_addr, ++consumed);   // V_j halves landed
                 if (!ok) return;
-                const int sb = j % NS;
                 if constexpr (C::MMA_WAITS_P) {
                     // P_j stored in both CTAs: waited here with try_wait, which suspends the
                     // warp (no issue slots taken from the softmax warp beside it)
-                    const uint32_t pb = PBAR(PB_P + sb);
-                    const uint32_t par = static_cast<uint32_t>(j / NS) & 1u;
+                    const uint32_t pb = PBAR(PB_P + (j & 1));
+                    const uint32_t par = (j >> 1) & 1;
                     if (!uniform(mbar_try_wait(pb, par))) {
                         const uint64_t t0 = global_timer_ns();
                         while (true) {
@@ -374,30 +357,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     }
                 }
                 tc_fence_after();
-                // PV_j reads P_j (over S_j) and adds into O, which the first PV starts fresh
-                const uint32_t p_tmem = tmem + static_cast<uint32_t>(sb) * BN;
-                const uint32_t o_tmem = tmem + C::O_COL;
+                // PV_j reads P_j (over S_j); two-group mode: it adds into O_{j&1}, and
+                // each accumulator starts fresh
+                const uint32_t p_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
+                const uint32_t o_tmem = tmem + O_COL + (C::DUAL ? static_cast<uint32_t>((j & 1) * D) : 0u);
+                const uint32_t acc0 = (j < (C::DUAL ? 2 : 1)) ? 0u : 1u;
                 const uint64_t vd = slot_desc(v_desc0);
 #pragma unroll
                 for (int kb = 0; kb < BN / 16; ++kb)
                     mma_ts_pair_elect(o_tmem, p_tmem + static_cast<uint32_t>(kb) * 8u,
-                                      vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV,
-                                      (j > 0 || kb > 0) ? 1u : 0u);
+                                      vd + static_cast<uint64_t>((kb * 16 * 128) >> 4), IDESC_PV, kb == 0 ? acc0 : 1u);
                 tc_commit_pair_elect(PBAR(PB_EMPTY + slot), 0x3);
-                // The pipelined softmax waits for PV_{j-1} before a rescale of O; the other
-                // mode learns of it from the S barrier of the tile issued after it, or (for
-                // the last tile) from PB_OPREV.  The once-only barriers complete exactly
-                // once, so a parity-0 wait on them cannot be confused by a later phase.
-                if constexpr (C::PIPE) tc_commit_pair_elect(PBAR(PB_PVD + (j & 1)), 0x3);
-                if (!C::PIPE && j == n_tiles - 2) tc_commit_pair_elect(PBAR(PB_OPREV), 0x3);
+                // Each O barrier completes exactly once, so a parity-0 wait on it cannot
+                // be confused by a later phase.
+                if (!C::DUAL && j == n_tiles - 2) tc_commit_pair_elect(PBAR(PB_OPREV), 0x3);
                 if (j == n_tiles - 1) tc_commit_pair_elect(PBAR(PB_OLAST), 0x3);
                 next_slot();
             };
-            for (int i = 0; i < NS && i < n_tiles && ok; ++i) issue_s(i);
+            if (ok) issue_s(0);
+            if (ok && n_tiles > 1) issue_s(1);
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
                 issue_pv(j);
-                if (ok && j + NS < n_tiles) issue_s(j + NS);
+                if (ok && j + 2 < n_tiles) issue_s(j + 2);
             }
             tc_commit_pair_elect(PBAR(PB_DRAIN), 0x1);
             __syncwarp();
@@ -406,255 +388,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
         __syncwarp();
     } else if (warp < C::SM_WARPS) {
         // ================================================================ softmax (both CTAs)
-        // Thread t of warps 0-3 owns query row q0 + t (TMEM lane t).
-        const int r = tid;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // Thread t of warpgroup w owns query row q0 + t % 128 (TMEM lane t % 128).  Two-group
+        // mode: group w takes the key tiles j = w (mod 2) with its own running max, row sum
+        // and O accumulator O_w, and the two partial results are merged exactly at the end
+        // (the log-sum-exp rule of split-KV); otherwise group 0 takes every tile.
+        constexpr bool DUAL = C::DUAL;
+        const int wg = warp >> 2;
+        const int r = tid & 127;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t o_col = O_COL + (DUAL ? static_cast<uint32_t>(wg * D) : 0u);
         const float sl2 = p.scale_log2;
-        float m_ref = -INFINITY;   // reference max, log2 domain
-        float l_sum = 0.0f;        // row sum relative to m_ref
+        const bool pos_scale = sl2 > 0.0f;
+        float m_ref = -INFINITY;
+        float l_sum = 0.0f;
         bool ok = true;
-        auto wait_fast = [&](uint32_t bar, uint32_t parity) -> bool {
-            if (mbar_test_wait(bar, parity)) return true;   // normally complete: no call
-            return wait_bar(bar, parity, abort_flag, wlim);
-        };
-        // P_j stored over S_j in this CTA: one arrival per warp on the leader's barrier
-        auto announce_p = [&](int sb) {
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(mapa_shared(PBAR(PB_P + sb), 0));
-        };
-        if constexpr (C::PIPE) {
-            // Pipelined mode.  A tile's work runs in four quarters of 32 columns.  Entering
-            // tile j the warp holds columns 0-63 of S_j (prepared) and the maximum of S_j.
-            // Loads are issued a half tile ahead of their use: columns 64-127 of S_j and
-            // 0-63 of S_{j+1} before the exponentials of quarters 0 and 1, columns 64-127 of
-            // S_{j+1} before quarter 2; the maximum of S_{j+1} is taken during quarters 2
-            // and 3.  The last two tiles (the masked maximum of the last tile, then the
-            // masked last tile without a next one) run separate copies of the tile body.
-            //
-            // Scores of one 32-column chunk (float bits, in place), starting at column col0:
-            // a zero or negative scale is applied here so that the maximum is taken over the
-            // scaled scores; in a masked tile the columns before `lo` are not this tile's
-            // keys and become -inf (by selection).
-            auto prep = [&](auto masked_t, uint32_t (&t)[32], int col0, int lo) {
-                constexpr bool MASKED = decltype(masked_t)::value;
-                if constexpr (MASKED || !POS) {
+        int seen = 0;   // tiles this group has processed
+#pragma unroll 1
+        for (int j = DUAL ? wg : 0; j < n_tiles; j += DUAL ? 2 : 1) {
+            // Two-group mode: S_j was issued after PV_{j-2}, the last PV into O_w before
+            // this tile, and its commit completes after every earlier MMA: from here on O_w
+            // is quiescent until PV_j, which needs this tile's P.
+            ok = __all_sync(0xffffffffu, wait_bar(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
+            uint32_t raw[BN];
+            tmem_ld128_wait(s_addr, raw);
+            float x[BN];
+            const int lo = (j == n_tiles - 1) ? last_lo : 0;   // columns [0, lo) are not this tile's keys
+            if (lo > 0) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float x = __uint_as_float(t[e]);
-                        if constexpr (!POS) x *= sl2;
-                        if constexpr (MASKED) x = (col0 + e < lo) ? -INFINITY : x;
-                        t[e] = __float_as_uint(x);
-                    }
-                }
-            };
-            using t_ = std::true_type;
-            using f_ = std::false_type;
-            uint32_t xl0[32], xl1[32];   // columns 0-31 and 32-63 of the current tile, prepared
-            uint32_t yl0[32], yl1[32];   // the same of the next tile, loaded during this one
-            float mx = -INFINITY;        // maximum of the current tile's prepared scores
-            if (n_tiles > 0) {
-                ok = __all_sync(0xffffffffu, wait_fast(PBAR(PB_S + 0), 0));
-                if (ok) {
-                    tc_fence_after();
-                    uint32_t t2[32], t3[32];
-                    tmem_ld32_nowait(tmem + lane_base, xl0);
-                    tmem_ld32_nowait(tmem + lane_base + 32, xl1);
-                    tmem_ld32_nowait(tmem + lane_base + 64, t2);
-                    tmem_ld32_nowait(tmem + lane_base + 96, t3);
-                    tmem_wait_ld_dep(xl0, xl1, t2, t3);
-                    if (n_tiles == 1) {
-                        prep(t_{}, xl0, 0, last_lo);
-                        prep(t_{}, xl1, 32, last_lo);
-                        prep(t_{}, t2, 64, last_lo);
-                        prep(t_{}, t3, 96, last_lo);
-                    } else {
-                        prep(f_{}, xl0, 0, 0);
-                        prep(f_{}, xl1, 32, 0);
-                        prep(f_{}, t2, 64, 0);
-                        prep(f_{}, t3, 96, 0);
-                    }
-                    mx = fmaxf(fmaxf(chunk_max32(xl0), chunk_max32(xl1)), fmaxf(chunk_max32(t2), chunk_max32(t3)));
-                }
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(raw[c]);
             }
-            int j = 0;
-            uint32_t buf = 0;     // j % 3
-            uint32_t par_n = 0;   // ((j + 1) / 3) & 1
-            const float mul = POS ? sl2 : 1.0f;
-            // One tile.  HN: a next tile exists; NM: the next tile is the masked last one;
-            // CM: this tile is the masked last one.
-            auto tile = [&](auto hn_t, auto nm_t, auto cm_t) -> bool {
-                constexpr bool HN = decltype(hn_t)::value;
-                const uint32_t nbuf = (buf == NS - 1) ? 0u : buf + 1u;
-                if (nbuf == 0) par_n ^= 1u;
-                if constexpr (HN) {
-                    // S_{j+1} was issued after PV_{j-2}; normally complete a tile ago
-                    if (!__all_sync(0xffffffffu, wait_fast(PBAR(PB_S + nbuf), par_n))) return false;
-                    tc_fence_after();
-                }
-                const float mt = mx * (POS ? sl2 : 1.0f);
-                float factor = 1.0f;
-                if (j == 0) {
-                    m_ref = mt;
-                } else if (__any_sync(0xffffffffu, mt > m_ref + RESCALE_LOG2)) {
-                    const float m_new = fmaxf(m_ref, mt);
-                    factor = fast_exp2(m_ref - m_new);
-                    m_ref = m_new;
-                    // PV_{j-1} must be complete before O is rescaled; PV_j needs this tile's
-                    // P.  The parity wait is unambiguous: S_j, issued after PV_{j-3}, is
-                    // complete, so the barrier of PV_{j-1}'s parity is at most one phase
-                    // behind.
-                    if (!__all_sync(0xffffffffu, wait_bar(PBAR(PB_PVD + ((j - 1) & 1)), ((j - 1) >> 1) & 1,
-                                                          abort_flag, wlim)))
-                        return false;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int oc = 0; oc < D / 32; ++oc) {
-                        uint32_t o[32];
-                        tmem_ld32_wait(tmem + lane_base + C::O_COL + oc * 32, o);
+            if (!pos_scale) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                        tmem_st32(tmem + lane_base + C::O_COL + oc * 32, o);
-                    }
-                }
-                const uint32_t s_addr = tmem + lane_base + buf * BN;
-                const uint32_t n_addr = tmem + lane_base + nbuf * BN;
-                const float2 mul_2 = make_float2(mul, mul);
-                const float2 neg_m2 = make_float2(-m_ref, -m_ref);
-                float2 sp[4];
+                for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
+            }
+            const float mx = row_max(x) * (pos_scale ? sl2 : 1.0f);   // three-input maxima
+            float factor = 1.0f;
+            bool rescale = false;
+            if (seen == 0) {
+                m_ref = mx;
+            } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
+                const float m_new = fmaxf(m_ref, mx);
+                factor = fast_exp2(m_ref - m_new);
+                m_ref = m_new;
+                rescale = true;
+            }
+            const float mul = pos_scale ? sl2 : 1.0f;
+            const float neg_m = -m_ref;
+            // p = 2^(x * mul - m): the scale-and-shift and the row sum in packed pairs
+            float2 sp[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
-                // p = 2^(x * mul - m) for 32 columns: packed scale-and-shift and row sum,
-                // bf16 pairs for the TMEM store of P over S_j
-                auto exp32 = [&](const uint32_t (&x)[32], uint32_t (&pk)[16]) {
+            for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
+            const float2 mul_2 = make_float2(mul, mul);
+            const float2 neg_m2 = make_float2(neg_m, neg_m);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 v = fma2(make_float2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])),
-                                              mul_2, neg_m2);
-                        const float p0 = fast_exp2(v.x);
-                        const float p1 = fast_exp2(v.y);
-                        sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                };
-                uint32_t xh0[32], xh1[32];
-                tmem_ld32_nowait(s_addr + 64, xh0);
-                tmem_ld32_nowait(s_addr + 96, xh1);
-                if constexpr (HN) {
-                    tmem_ld32_nowait(n_addr, yl0);
-                    tmem_ld32_nowait(n_addr + 32, yl1);
-                }
-                uint32_t pk0[16], pk1[16];
-                exp32(xl0, pk0);
-                tmem_st16_at(s_addr, pk0);   // P columns 0-15 over S columns 0-31, already read
-                exp32(xl1, pk1);
-                if constexpr (HN) tmem_wait_ld_dep(xh0, xh1, yl0, yl1);
-                else tmem_wait_ld_dep(xh0, xh1);
-                tmem_st16_at(s_addr + 16, pk1);
-                prep(cm_t, xh0, 64, last_lo);
-                prep(cm_t, xh1, 96, last_lo);
-                uint32_t m0[32], m1[32];
-                if constexpr (HN) {
-                    tmem_ld32_nowait(n_addr + 64, m0);
-                    tmem_ld32_nowait(n_addr + 96, m1);
-                }
-                uint32_t pk2[16], pk3[16];
-                exp32(xh0, pk2);
-                float mxn = -INFINITY;
-                if constexpr (HN) {
-                    prep(nm_t, yl0, 0, last_lo);
-                    prep(nm_t, yl1, 32, last_lo);
-                    mxn = fmaxf(chunk_max32(yl0), chunk_max32(yl1));
-                    tmem_wait_ld_dep(m0, m1);
-                }
-                tmem_st16_at(s_addr + 32, pk2);
-                exp32(xh1, pk3);
-                if constexpr (HN) {
-                    prep(nm_t, m0, 64, last_lo);
-                    prep(nm_t, m1, 96, last_lo);
-                    mxn = fmaxf(mxn, fmaxf(chunk_max32(m0), chunk_max32(m1)));
-                }
-                tmem_st16_at(s_addr + 48, pk3);
-                const float tile_sum =
-                    ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
-                l_sum = l_sum * factor + tile_sum;
-                announce_p(static_cast<int>(buf));
-                if constexpr (HN) {
-                    mx = mxn;
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        xl0[e] = yl0[e];
-                        xl1[e] = yl1[e];
-                    }
+                for (int e = 0; e < 16; ++e) {
+                    const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
+                    const float p0 = fast_exp2(y.x);
+                    const float p1 = fast_exp2(y.y);
+                    sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
-                buf = nbuf;
-                ++j;
-                return true;
-            };
-#pragma unroll 1
-            while (ok && j + 2 < n_tiles) ok = tile(t_{}, f_{}, f_{});
-            if (ok && j + 1 < n_tiles) ok = tile(t_{}, t_{}, f_{});   // the next tile is the last one
-            if (ok && j < n_tiles) ok = tile(f_{}, f_{}, t_{});       // the last tile
-        } else {
-            // Per tile: the S tile is loaded, its row maximum taken, then the exponentials.
-            const bool pos_scale = sl2 > 0.0f;
-#pragma unroll 1
-            for (int j = 0; j < n_tiles; ++j) {
-                ok = __all_sync(0xffffffffu, wait_bar(PBAR(PB_S + (j & 1)), (j >> 1) & 1, abort_flag, wlim));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t s_addr = tmem + lane_base + static_cast<uint32_t>(j & 1) * BN;
-                uint32_t raw[BN];
-                tmem_ld128_wait(s_addr, raw);
-                float x[BN];
-                const int lo = (j == n_tiles - 1) ? last_lo : 0;   // columns [0, lo) are not this tile's keys
-                if (lo > 0) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(raw[c]);
-                }
-                if (!pos_scale) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) x[c] = (c >= lo) ? x[c] * sl2 : -INFINITY;
-                }
-                const float mx = row_max(x) * (pos_scale ? sl2 : 1.0f);   // three-input maxima
-                float factor = 1.0f;
-                bool rescale = false;
-                if (j == 0) {
-                    m_ref = mx;
-                } else if (__any_sync(0xffffffffu, mx > m_ref + RESCALE_LOG2)) {
-                    const float m_new = fmaxf(m_ref, mx);
-                    factor = fast_exp2(m_ref - m_new);
-                    m_ref = m_new;
-                    rescale = true;
-                }
-                const float mul = pos_scale ? sl2 : 1.0f;
-                const float neg_m = -m_ref;
-                // p = 2^(x * mul - m): the scale-and-shift and the row sum in packed pairs
-                float2 sp[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) sp[t] = make_float2(0.0f, 0.0f);
-                const float2 mul_2 = make_float2(mul, mul);
-                const float2 neg_m2 = make_float2(neg_m, neg_m);
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 y = fma2(make_float2(x[cc * 32 + 2 * e], x[cc * 32 + 2 * e + 1]), mul_2, neg_m2);
-                        const float p0 = fast_exp2(y.x);
-                        const float p1 = fast_exp2(y.y);
-                        sp[e & 3] = add2(sp[e & 3], make_float2(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(s_addr + cc * 16, pk);
-                }
-                const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
-                l_sum = l_sum * factor + tile_sum;
-                if (rescale) {
+                tmem_st16(s_addr + cc * 16, pk);
+            }
+            const float tile_sum = ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
+            l_sum = l_sum * factor + tile_sum;
+            if (rescale) {
+                if constexpr (!DUAL) {
                     // PV_{j-1} is complete once S_{j+1} (issued after it) is; for the last
                     // tile the leader announces PV_{n-2} on its own barrier.
                     const bool w = (j + 1 < n_tiles)
@@ -663,17 +471,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     ok = __all_sync(0xffffffffu, w);
                     if (!ok) break;
                     tc_fence_after();
-#pragma unroll 1
-                    for (int oc = 0; oc < D / 32; ++oc) {
-                        uint32_t o[32];
-                        tmem_ld32_wait(tmem + lane_base + C::O_COL + oc * 32, o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                        tmem_st32(tmem + lane_base + C::O_COL + oc * 32, o);
-                    }
                 }
-                announce_p(j & 1);
+#pragma unroll 1
+                for (int oc = 0; oc < D / 32; ++oc) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tmem + lane_base + o_col + oc * 32, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                    tmem_st32(tmem + lane_base + o_col + oc * 32, o);
+                }
             }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(mapa_shared(PBAR(PB_P + (j & 1)), 0));
+            ++seen;
         }
         // ---- epilogue
         if (ok && n_tiles > 0) {
@@ -682,20 +494,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             ok = __all_sync(0xffffffffu, w);
             tc_fence_after();
         }
+        // Two-group mode: m = max_w m_w, f_w = 2^(m_w - m), l = sum_w l_w f_w,
+        // O = sum_w O_w f_w / l (a group with no tile has l_w = 0 and weight 0).
+        float f_own = 1.0f, f_other = 0.0f, m_row = m_ref, l_row = l_sum;
+        bool own_has = n_tiles > 0, other_has = false;
+        if constexpr (DUAL) {
+            float* xch = reinterpret_cast<float*>(sKV + C::NSLOTS * C::SLOT + C::CTRL);   // [2][max, sum][128]
+            xch[(wg * 2 + 0) * 128 + r] = m_ref;
+            xch[(wg * 2 + 1) * 128 + r] = l_sum;
+            named_barrier_sync(XCH_ID, 32 * C::SM_WARPS);
+            const float m_o = xch[((wg ^ 1) * 2 + 0) * 128 + r];
+            const float l_o = xch[((wg ^ 1) * 2 + 1) * 128 + r];
+            own_has = l_sum > 0.0f;
+            other_has = l_o > 0.0f;
+            m_row = own_has ? (other_has ? fmaxf(m_ref, m_o) : m_ref) : m_o;
+            f_own = own_has ? fast_exp2(m_ref - m_row) : 0.0f;
+            f_other = other_has ? fast_exp2(m_o - m_row) : 0.0f;
+            l_row = l_sum * f_own + l_o * f_other;
+        }
         const int row = q0 + r;
         const bool in_range = row < p.Tq;
         const bool have = n_tiles > 0;
-        const float inv_l = have ? 1.0f / l_sum : 0.0f;
-        const float lse_val = have ? (m_ref + log2f(l_sum)) * LN2 : -INFINITY;
+        const float inv_l = have ? 1.0f / l_row : 0.0f;
+        const float lse_val = have ? (m_row + log2f(l_row)) * LN2 : -INFINITY;
         const long long BH = static_cast<long long>(p.B) * p.H;
+        const uint32_t o_col_other = O_COL + static_cast<uint32_t>((wg ^ 1) * D);
+        // two-group mode: group w writes the 32-column chunks oc = w (mod 2)
 #pragma unroll 1
-        for (int oc = 0; oc < D / 32; ++oc) {
+        for (int oc = DUAL ? wg : 0; oc < D / 32; oc += DUAL ? 2 : 1) {
             uint32_t o[32];
-            if (have) {
-                tmem_ld32_wait(tmem + lane_base + C::O_COL + oc * 32, o);
+            if (have && own_has) {
+                tmem_ld32_wait(tmem + lane_base + o_col + oc * 32, o);
+                if constexpr (DUAL) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_own);
+                }
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = 0u;
+            }
+            if (DUAL && have && other_has) {
+                uint32_t o2[32];
+                tmem_ld32_wait(tmem + lane_base + o_col_other + oc * 32, o2);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[e] = __float_as_uint(fmaf(__uint_as_float(o2[e]), f_other, __uint_as_float(o[e])));
             }
             if (!in_range) continue;
             if constexpr (SPLIT) {
@@ -719,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 }
             }
         }
-        if (in_range) {
+        if (in_range && wg == 0) {
             if constexpr (SPLIT) {
                 p.part_lse[(static_cast<long long>(split) * BH + bh) * p.Tq + row] = lse_val;
             } else if (p.lse != nullptr) {

@@ -50,16 +50,3 @@ __device__ __forceinline__ float row_max(const float (&x)[N]) {
     return fmaxf(max3f(m[0], m[1], m[2]), max3f(max3f(m[3], m[4], m[5]), m[6], m[7]));
 }
 
-// Maximum of the 32 values of one chunk (float bits): four chains of three-input maxima.
-__device__ __forceinline__ float chunk_max32(const uint32_t (&t)[32]) {
-    float m[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int b = c * 8;
-        m[c] = max3f(__uint_as_float(t[b]), __uint_as_float(t[b + 1]), __uint_as_float(t[b + 2]));
-        m[c] = max3f(m[c], __uint_as_float(t[b + 3]), __uint_as_float(t[b + 4]));
-        m[c] = max3f(m[c], __uint_as_float(t[b + 5]), __uint_as_float(t[b + 6]));
-        m[c] = fmaxf(m[c], __uint_as_float(t[b + 7]));
-    }
-    return fmaxf(max3f(m[0], m[1], m[2]), m[3]);
-}
