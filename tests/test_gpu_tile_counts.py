@@ -1,13 +1,14 @@
 """GPU parity at every small key-tile count, against the fp64 oracle.
 
-The CTA-pair kernel keeps S_0 .. S_{NS-1} in TMEM (NS = 3 at head dim 128, 2 at 256).
-At head dim 128 its softmax takes the row maximum of tile j + 1 during tile j and runs
-separate code for the tile whose successor is the masked last tile and for the last tile
-itself; with fewer tiles than S buffers, the MMA warp issues fewer S tiles up front.
-This sweeps 1 to 5 key tiles (all-full and partial last tiles, a last tile of one valid
-key, a prefix ending one key into a tile), positive, zero and negative scales (the sign
-of the scale selects a separate specialisation), at head dims 128 and 256, single pass
-and split-KV, with K/V padding set to NaN so any read of it would show.
+The CTA-pair kernel issues S_0 and S_1 up front, then PV_j and S_{j+2} per tile, with
+P_j stored over S_j. At head dim 128 two softmax warpgroups take alternate key tiles
+(group 1 gets no tile at all when there is one) and merge their partial results at the
+end; the masked last tile belongs to either group. With fewer tiles than S buffers the
+MMA warp issues fewer S tiles up front. This sweeps 1 to 5 key tiles (all-full and
+partial last tiles, a last tile of one valid key, a prefix ending one key into a tile),
+positive, zero and negative scales (the sign of the scale selects a separate
+specialisation), at head dims 128 and 256, single pass and split-KV, with K/V padding
+set to NaN so any read of it would show.
 """
 import pytest
 import torch
