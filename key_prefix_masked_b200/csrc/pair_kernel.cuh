@@ -172,10 +172,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             tma_prefetch_map(&tm_v);
             if (leader) mbar_arrive_expect_tx(PBAR(PB_Q), 2 * C::Q_BYTES);
             const uint32_t lq = mapa_shared(PBAR(PB_Q), 0);
-            // Q is read once: evict it first.  Every pair of the head streams the head's K/V:
-            // keep those lines in L2 ahead of Q and of the output stream.
+            // Q is read once: evict it first.  Every pair of the head streams the head's K/V,
+            // so half of its lines are kept in L2 ahead of Q and of the output stream.  Half,
+            // not all: where the resident clusters span two heads whose K/V together exceed
+            // L2 (2 x 102 MB at 100000 keys, D=256), protected lines of both heads would
+            // evict one another; the protected halves of two heads fit.
             const uint64_t pol_q = l2_policy_evict_first();
-            const uint64_t pol_kv = l2_policy_evict_last();
+            const uint64_t pol_kv = l2_policy_evict_last_half();
 #pragma unroll
             for (int blk = 0; blk < C::NBLK; ++blk)
                 tma_load_4d_pair_hint(sQ_addr + blk * (C::ROWS * 128), &tm_q, blk * 64, q0, h, b, lq, pol_q);
@@ -208,8 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                     phase ^= 1u;
                 }
             };
-            item(true, 0);
-            if (n_tiles > 1) item(true, 1);
+            for (int i = 0; i < 2 && i < n_tiles; ++i) item(true, i);
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
                 item(false, j);
@@ -244,10 +246,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
             auto publish = [&]() {
                 if (ok) st_release_smem(seq_addr, ++seq);
             };
-            item();  // K_0
-            publish();
-            if (n_tiles > 1) {
-                item();  // K_1
+            for (int i = 0; i < 2 && i < n_tiles; ++i) {
+                item();  // K_i
                 publish();
             }
 #pragma unroll 1
@@ -374,8 +374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<D>::THREADS,
                 if (j == n_tiles - 1) tc_commit_pair_elect(PBAR(PB_OLAST), 0x3);
                 next_slot();
             };
-            if (ok) issue_s(0);
-            if (ok && n_tiles > 1) issue_s(1);
+            for (int i = 0; i < 2 && i < n_tiles && ok; ++i) issue_s(i);
 #pragma unroll 1
             for (int j = 0; j < n_tiles && ok; ++j) {
                 issue_pv(j);

@@ -252,9 +252,11 @@ __device__ __forceinline__ void tma_load_4d_pair_hint(uint32_t dst, const void* 
         : "memory");
 }
 // L2 policies: lines read under evict_last stay in L2 ahead of normal and evict_first lines.
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+// The fractional form gives evict_last to half of the lines an access covers (chosen by
+// address) and leaves the priority of the other half unchanged.
+__device__ __forceinline__ uint64_t l2_policy_evict_last_half() {
     uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+    asm volatile("createpolicy.fractional.L2::evict_last.L2::evict_unchanged.b64 %0, 0.5;\n" : "=l"(pol));
     return pol;
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
