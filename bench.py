@@ -266,7 +266,7 @@ class Problem:
         # work done by this rank (the whole job's work is flops_total in the sharded modes)
         rows = self.r1 - self.r0
         self.flops_rank = float(sum(4.0 * w.H * rows * n * w.D for n in self.kv_list))
-        self.flops_job = self.flops_total if (shard in ("queries", "keys") and world > 1) else self.flops_total * world
+        self.flops_job = job_flops(w, case["kv_len_list"], world, shard)
         B, H, D = w.B, w.H, w.D
         Tq_l = self.q.shape[2]
         self.out = torch.empty((B, H, Tq_l, D), dtype=torch.bfloat16, device=dev)
@@ -359,6 +359,43 @@ def l2_note(flushed: bool):
             "events; value from per-step events")
 
 
+def input_bytes(w, rank, world, shard) -> int:
+    """Bytes of q, k and v that one rank holds (its shard)."""
+    from key_prefix_masked_b200 import sharded
+    rows, keys = w.Tq, w.Tk
+    if world > 1 and shard == "queries":
+        r0, r1 = sharded.query_rows(w.Tq, rank, world)
+        rows = r1 - r0
+    elif world > 1 and shard == "keys":
+        k0, k1 = sharded.key_bounds(w.Tk, rank, world)
+        keys = k1 - k0
+    return 2 * w.B * w.H * w.D * (rows + 2 * keys)
+
+
+def needs_flush(w, rank, world, shard) -> bool:
+    return input_bytes(w, rank, world, shard) < 2 * L2_BYTES
+
+
+def job_flops(w, kv_len_list, world, shard) -> float:
+    total = workload_flops(w, kv_len_list)
+    return total if (shard in ("queries", "keys") and world > 1) else total * world
+
+
+SCALING = {"queries": "strong", "keys": "strong", "replicas": "weak", "single": "weak"}
+PARALLELISM = {"queries": "query rows sharded x{n} (no exchange)",
+               "keys": "key slots sharded x{n} (all-gather of partials, exact combine)",
+               "replicas": "replicas x{n}", "single": "single GPU"}
+
+
+def workload_config(w, case, args, world, shard, flushed):
+    """The `config` object of a line; both arms build it here, so they name the same work."""
+    return {**w.describe(),
+            "kv_len": case["kv_len_list"] if len(case["kv_len_list"]) <= 8 else "ragged",
+            "scale": case["scale"], "flops_per_step": job_flops(w, case["kv_len_list"], world, shard),
+            "l2": l2_note(flushed),
+            **({"split_mode": args.split_mode} if w.num_splits > 1 else {})}
+
+
 def measure(kp, name, args, rank, world, shard, steps, min_ms=0.0):
     """Device-timed measurement of one workload: (record fields, problem)."""
     w = synth.WORKLOADS[name]
@@ -371,7 +408,8 @@ def measure(kp, name, args, rank, world, shard, steps, min_ms=0.0):
     if st != kp.ATTN_OK:
         raise RuntimeError(f"{name}: device status after warm-up: {kp.status_string(st)}")
     in_bytes = sum(t.numel() * t.element_size() for t in (prob.q, prob.k, prob.v))
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
+    assert in_bytes == input_bytes(w, rank, world, shard), "shard shapes"
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if needs_flush(w, rank, world, shard) else None
     step_ms, total_ms, clocks, steps = device_timed(prob, steps, world, flush, torch.cuda.current_device(), min_ms)
     st = kp.device_status()
     if st != kp.ATTN_OK:
@@ -389,10 +427,7 @@ def measure(kp, name, args, rank, world, shard, steps, min_ms=0.0):
     achieved = kern_flops / (statistics.mean(kern_ms) * 1e-3) / 1e12
     rec = {
         "value": round(value, 2), "ms_per_step": round(ms_per_step, 4), "steps": steps,
-        "config": {**w.describe(), "kv_len": prob.case["kv_len_list"] if len(prob.case["kv_len_list"]) <= 8
-                   else "ragged", "scale": prob.scale, "flops_per_step": prob.flops_job,
-                   "l2": l2_note(flush),
-                   **({"split_mode": args.split_mode} if prob.splits else {})},
+        "config": workload_config(w, prob.case, args, world, shard, flush),
         "roofline": roofline_entry(w, name, achieved, clocks, prob.splits),
         "gpu_launches": prob.launches_per_step * steps,
         "clocks": clocks,
@@ -458,10 +493,8 @@ def run_ours(args, rank, world):
     shard = resolve_shard(args.shard, w) if world > 1 else "single"
     head, prob = measure(kp, args.workload, args, rank, world, shard, args.steps)
     e2e = run_e2e(kp, prob, args, world)
-    scaling = {"queries": "strong", "keys": "strong", "replicas": "weak", "single": "weak"}[shard]
-    parallelism = {"queries": f"query rows sharded x{world} (no exchange)",
-                   "keys": f"key slots sharded x{world} (all-gather of partials, exact combine)",
-                   "replicas": f"replicas x{world}", "single": "single GPU"}[shard]
+    scaling = SCALING[shard]
+    parallelism = PARALLELISM[shard].format(n=world)
     rec = {
         "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world,
         "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
@@ -674,6 +707,7 @@ def run_reference(args, rank, world):
     rows of the same workload."""
     import oracle
     w = synth.WORKLOADS[args.workload]
+    shard = resolve_shard(args.shard, w) if world > 1 else "single"
     case = synth.make_inputs(w, device="cpu", seed=args.seed)
     cores = oracle.num_threads()
     per_step_rows = _rows_for(w, case, args.cpu_seconds / max(args.steps + args.warmup, 1))
@@ -689,9 +723,10 @@ def run_reference(args, rank, world):
     return {
         "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot / args.steps * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {**w.describe(), "kv_len": case["kv_len_list"]
-                                        if len(case["kv_len_list"]) <= 8 else "ragged"},
+        "higher_is_better": True, "scaling": SCALING[shard], "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {**workload_config(w, case, args, world, shard, needs_flush(w, 0, world, shard)),
+                   "parallelism": PARALLELISM[shard].format(n=world)},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle",

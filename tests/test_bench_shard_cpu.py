@@ -80,6 +80,8 @@ res["q_lse_ninf_same"] = bool(np.array_equal(np.isneginf(got_l), np.isneginf(ref
 fin = np.isfinite(ref_l)
 res["q_err_lse"] = float(np.abs(got_l[fin] - ref_l[fin]).max())
 res["q_flops_job"] = pq.flops_job
+res["q_in_bytes_ok"] = bench.input_bytes(wq, rank, world, "queries") == sum(
+    t.numel() * t.element_size() for t in (pq.q, pq.k, pq.v))
 res["q_flops_total"] = pq.flops_total
 # split-KV workload, key-sharded: 700 key slots -> blocks of 384 and 316 (3 and 3 tiles);
 # element 1's prefix (200) ends inside rank 0's block
@@ -94,6 +96,8 @@ res["k_chunks"] = pk.c_local
 res["k_err_out"] = float(np.abs(pk.out.float().numpy() - ref_o).max())
 res["k_err_lse"] = float(np.abs(pk.lse.numpy() - ref_l).max())
 res["k_flops_rank"] = pk.flops_rank
+res["k_in_bytes_ok"] = bench.input_bytes(wk, rank, world, "keys") == sum(
+    t.numel() * t.element_size() for t in (pk.q, pk.k, pk.v))
 res["k_flops_total"] = pk.flops_total
 print(json.dumps({"rank": rank, **res}), flush=True)
 dist.destroy_process_group()
@@ -130,6 +134,8 @@ def test_two_gloo_ranks_shard_queries_and_keys(tmp_path):
         assert [tuple(r) for r in o["q_ranges"]] == [(0, 19), (19, 37)]
         assert o["q_err_out"] < 1e-2 and o["q_err_lse"] < 1e-6 and o["q_lse_ninf_same"]
         assert o["q_flops_job"] == o["q_flops_total"]
+        # the L2-flush decision and the configs both arms print use these shard sizes
+        assert o["q_in_bytes_ok"] and o["k_in_bytes_ok"]
         # key sharding: every rank holds the exact combined result
         assert o["k_err_out"] < 1e-2 and o["k_err_lse"] < 1e-6
         assert o["k_chunks"] == 2
@@ -152,3 +158,22 @@ def test_shard_blocks_cover_every_row_and_key_once():
         assert ks[0][0] == 0 and ks[-1][1] == Tk
         assert all(a[1] == b[0] and a[1] % 128 == 0 for a, b in zip(ks, ks[1:]))
     assert sharded.shard_kv_len([650, 200, 0, 700], 384, 700) == [266, 0, 0, 316]
+
+
+def test_reference_arm_names_the_same_config():
+    """The reference arm's `config` is the one the GPU arm prints for the same workload,
+    so the two lines name the same work (its value comes from a bounded oracle sample)."""
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    for name in ("tiny", "unmasked_8v"):
+        w = synth.WORKLOADS[name]
+        args = types.SimpleNamespace(workload=name, seed=0, cpu_seconds=0.2, steps=1, warmup=3,
+                                     shard="auto", split_mode="separate")
+        rec = bench.run_reference(args, 0, 1)
+        case = synth.make_inputs(w, device="cpu", seed=0)
+        ours = {**bench.workload_config(w, case, args, 1, "single", bench.needs_flush(w, 0, 1, "single")),
+                "parallelism": bench.PARALLELISM["single"].format(n=1)}
+        assert rec["config"] == ours
+        assert rec["scaling"] == "weak" and rec["impl"] == "reference"
