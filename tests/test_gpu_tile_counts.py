@@ -1,14 +1,15 @@
 """GPU parity at every small key-tile count, against the fp64 oracle.
 
-The CTA-pair kernel issues S_0 and S_1 up front, then PV_j and S_{j+2} per tile, with
-P_j stored over S_j. At head dim 128 two softmax warpgroups take alternate key tiles
-(group 1 gets no tile at all when there is one) and merge their partial results at the
-end; the masked last tile belongs to either group. With fewer tiles than S buffers the
-MMA warp issues fewer S tiles up front. This sweeps 1 to 5 key tiles (all-full and
+Both kernels issue S_0 and S_1 up front, then PV_j and S_{j+2} per tile (the single-CTA
+kernel's two-group mode at head dims 32 and 64: S_2 before PV_0, then S_{j+3}, with P in
+buffers of its own). Two softmax warpgroups take alternate key tiles at head dims 32, 64
+and 128 (group 1 gets no tile at all when there is one) and merge their partial results
+at the end; the masked last tile belongs to either group. With fewer tiles than S buffers
+the MMA warp issues fewer S tiles up front. This sweeps 1 to 5 key tiles (all-full and
 partial last tiles, a last tile of one valid key, a prefix ending one key into a tile),
 positive, zero and negative scales (the sign of the scale selects a separate
-specialisation), at head dims 128 and 256, single pass and split-KV, with K/V padding
-set to NaN so any read of it would show.
+specialisation), at every head dim, single pass and split-KV, with K/V padding set to
+NaN so any read of it would show.
 """
 import pytest
 import torch
@@ -35,7 +36,7 @@ KV_LENS = (128, 256, 384, 512, 640, 1, 129, 300, 385, 600, 513, 639)
 SCALES = (None, 0.0, -0.04)
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("scale", SCALES)
 def test_tile_counts_single_pass(kp, D, scale):
     B = len(KV_LENS)
@@ -50,7 +51,7 @@ def test_tile_counts_single_pass(kp, D, scale):
     assert_lse_close(lse, ref_lse, what=f"lse D={D} scale={sc}")
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_tile_counts_split(kp, D):
     # chunks of 256 keys (2 tiles): chunk-local tile counts of 0, 1 and 2, ragged ends
     B = len(KV_LENS)
