@@ -667,9 +667,18 @@ def _rows_for(w, case, seconds: float) -> int:
     return max(1, min(w.Tq, int(n * seconds / max(dt, 1e-4))))
 
 
+def host_oracle():
+    """The oracle module, set to run on every host core this process may use.  (torchrun
+    starts each rank with OMP_NUM_THREADS=1; the oracle is timed on rank 0 alone, so it
+    takes the cores back.)"""
+    import oracle
+    oracle.set_num_threads(len(os.sched_getaffinity(0)))
+    return oracle
+
+
 def oracle_full(case, w):
     """The oracle over the whole problem (every query row), timed on the host cores."""
-    import oracle
+    oracle = host_oracle()
     t = time.perf_counter()
     _oracle_rows(case, case["q"].cpu())
     dt = time.perf_counter() - t
@@ -681,7 +690,7 @@ def oracle_full(case, w):
 def oracle_extrapolated(case, w, n_rows=32):
     """The oracle on n_rows random query rows (all their valid keys), and the whole
     problem's time extrapolated linearly in rows x kv_len."""
-    import oracle
+    oracle = host_oracle()
     rows, dt, flops = _oracle_sample(w, case, n_rows, seed=3)
     full = workload_flops(w, case["kv_len_list"])
     return {"kind": "oracle, sampled rows", "sample": f"{len(rows)} random query rows x {w.H} heads",
@@ -690,7 +699,7 @@ def oracle_extrapolated(case, w, n_rows=32):
 
 
 def cpu_baseline(w, case, target_s: float):
-    import oracle
+    oracle = host_oracle()
     cores = oracle.num_threads()
     rows, dt, flops = _oracle_sample(w, case, _rows_for(w, case, target_s), seed=1)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
@@ -705,7 +714,7 @@ def cpu_baseline(w, case, target_s: float):
 def run_reference(args, rank, world):
     """The oracle timed on the host cores: each step evaluates a bounded sample of query
     rows of the same workload."""
-    import oracle
+    oracle = host_oracle()
     w = synth.WORKLOADS[args.workload]
     shard = resolve_shard(args.shard, w) if world > 1 else "single"
     case = synth.make_inputs(w, device="cpu", seed=args.seed)

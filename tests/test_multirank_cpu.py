@@ -69,3 +69,16 @@ def test_reference_arm_runs_on_host_cores():
     rec = json.loads(out.stdout.strip().splitlines()[-1])
     assert rec["impl"] == "reference" and rec["value"] > 0 and rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["higher_is_better"] is True
+
+
+def test_reference_arm_takes_the_host_cores_back_from_torchrun_s_default():
+    """torchrun starts every rank with OMP_NUM_THREADS=1; the reference arm (rank 0 alone)
+    still times the oracle on every core the process may use."""
+    import json
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "2", "--warmup", "3", "--cpu-seconds", "0.5"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr
+    rec = json.loads(out.stdout.strip().splitlines()[-1])
+    assert rec["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
