@@ -459,7 +459,11 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     } else if (warp == C::WARP_MMA) {
         // ================================================================ MMA issuer (one warp)
         // Two readiness events per tile, published by the relay warp: "P_j stored and
-        // V_j landed" and "K_{j+2} landed".  Between them the 8 PV and 16 S MMAs of a
+        // V_j landed" and "K_{j+2} landed" (two-group mode: "S_{j+1} read out and K_{j+3}
+        // landed" and "V_j landed", and this warp waits for "P_j stored" itself, with a
+        // suspending try_wait: the relay's wake-up and this warp's poll had put ~850
+        // cycles between the last P arrival and PV_j; same-box A/B +4.5 % at N 13622 and
+        // 7784, +2.2 % at N 31136).  Between them the 8 PV and 16 S MMAs of a
         // tile are issued as straight-line code from precomputed descriptors, so the
         // tensor pipe's queue stays fed (the tile's MMA mix alone runs at the tensor
         // peak; the issuing code's overhead is what decides the rate).  The whole warp
@@ -512,6 +516,23 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     }
                 }
                 return __shfl_sync(0xffffffffu, ok_ev ? 1 : 0, 0) != 0;
+            };
+            auto uniform = [&](bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; };
+            // a barrier the softmax warps arrive on, waited with try_wait (suspends the warp)
+            auto wait_arrivals = [&](uint32_t bar, uint32_t par) -> bool {
+                if (uniform(mbar_try_wait(bar, par))) return true;
+                const uint64_t t0 = global_timer_ns();
+                while (true) {
+                    if (uniform(mbar_try_wait(bar, par))) return true;
+                    if (uniform(*abort_flag != 0)) return false;
+                    if (uniform(global_timer_ns() - t0 > wlim)) {
+                        if (lane == 0) {
+                            *abort_flag = 1;
+                            atomicOr(&g_attn_status, STATUS_TIMEOUT);
+                        }
+                        return false;
+                    }
+                }
             };
             auto issue_s = [&](int j) {
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(j & 1) * BN;
@@ -594,7 +615,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         tc_fence_after();
                         issue_s(j + 3);
                     }
-                    ok = next_event();   // P_j stored and V_j landed
+                    ok = next_event();   // V_j landed
+                    if (!ok) break;
+                    ok = wait_arrivals(BAR(BAR_P + (j & 1)), (j >> 1) & 1);   // P_j stored
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(j);
@@ -626,7 +649,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         // and publishes one completed event per MMA batch with a release store: K_0,
         // K_1, then per tile j "P_j + V_j" and "K_{j+2}"; the MMA thread acquires it.
         // Two-group mode: K_0, K_1, "S_0 read + K_2", then per tile j "S_{j+1} read +
-        // K_{j+3}" and "P_j + V_j".
+        // K_{j+3}" and "V_j" (the MMA thread waits for P_j itself).
         if (lane == 0 && n_tiles > 0) {
             int gi = 0;
             uint32_t phase = 0, seq = 0;
@@ -661,8 +684,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         s_read(j + 1);
                         relay_s();
                     }
-                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();   // V_j first: usually landed
-                    ok = ok && wait_bar(BAR(BAR_P + (j & 1)), (j >> 1) & 1, abort_flag, wlim);
+                    for (int g = 0; g < C::VCH / C::GRP; ++g) group();   // V_j
                     publish();
                 }
             } else {
