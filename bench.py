@@ -637,9 +637,11 @@ def traffic_from_profile(workload: str, kernel: str):
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.json")
     try:
         with open(path) as f:
-            return json.load(f).get("dram_bytes_per_launch")
+            rec = json.load(f)
     except (OSError, ValueError):
         return None
+    # null once the kernel has changed since the counters were taken
+    return rec.get("dram_bytes_per_launch") if rec.get("current", True) else None
 
 
 # ------------------------------------------------------------------ CPU baseline / reference arm
