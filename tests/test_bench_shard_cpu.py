@@ -177,3 +177,18 @@ def test_reference_arm_names_the_same_config():
                 "parallelism": bench.PARALLELISM["single"].format(n=1)}
         assert rec["config"] == ours
         assert rec["scaling"] == "weak" and rec["impl"] == "reference"
+
+
+def test_traffic_of_a_changed_kernel_is_null(tmp_path, monkeypatch):
+    """A committed traffic summary counts only while it was taken on the current kernel."""
+    import json as _json
+    sys.path.insert(0, ROOT)
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "k_w_traffic.json").write_text(_json.dumps({"dram_bytes_per_launch": 123}))
+    (prof / "k_old_traffic.json").write_text(_json.dumps({"dram_bytes_per_launch": 456, "current": False}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profile("w", "k") == 123
+    assert bench.traffic_from_profile("old", "k") is None
+    assert bench.traffic_from_profile("missing", "k") is None
